@@ -1,0 +1,22 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a) and the built library")
+
+
+@pytest.fixture(scope="session")
+def cuda_lib():
+    """The built CUDA library; GPU tests fail loudly when it is missing."""
+    import torch
+    import paged_kv_cache_325_b200 as pa
+    assert torch.cuda.is_available(), "GPU test collected without a CUDA device"
+    pa.load_library()
+    return pa

@@ -1,0 +1,217 @@
+/*
+ * pa.h -- C ABI of the B200 (sm_100a) paged-KV attention library (libpagedattn.so).
+ *
+ * Three operations make up one attention layer call of a paged-KV inference
+ * engine of the nano-vllm kind:
+ *
+ *   pa_store_kv        write this step's new K/V rows into the block-paged cache
+ *   pa_decode          one query token per sequence attends to its whole context
+ *   pa_prefill_varlen  the new (uncached) tokens of each prompt attend causally
+ *                      to the cached prefix plus themselves
+ *
+ * The call order follows the attention forward of the nano-vllm walkthrough
+ * (xingyun3d.csdn.net, section seven "后端执行（cuda 算子）"): store first, then
+ * prefill or decode on the same stream.  Argument names follow the per-step
+ * context object of the same page (section eight "序列与上下文"): slot_mapping,
+ * context_lens, block_tables, cu_seqlens_q/k, max_seqlen_q/k.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE memory owned by the caller.  The library
+ *    never allocates, frees or retains them and keeps no state between calls
+ *    other than a per-device cache of kernel attributes.
+ *  - Element type: K, V, Q and outputs are bfloat16 (passed as void*); every
+ *    index array is int32.
+ *  - Cache layout: k_cache and v_cache are [num_blocks, block_size,
+ *    num_kv_heads, head_dim], contiguous, 16-byte aligned.  Token p of a
+ *    sequence lives in slot block_table[s][p / block_size] * block_size +
+ *    p % block_size (block index and in-block offset, gsyq.cn nano-vLLM
+ *    article, section 4.1).
+ *  - Supported shapes: head_dim in {64, 128}; block_size a power of two in
+ *    [16, 256]; num_q_heads a multiple of num_kv_heads with
+ *    num_q_heads / num_kv_heads <= 16.  Anything else returns
+ *    PA_ERR_UNSUPPORTED.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *    entry point is asynchronous: it validates its host-side arguments
+ *    synchronously, enqueues its kernels and returns.
+ *  - Host-side errors (bad scalars, null or misaligned pointers, a workspace
+ *    that is too small) return an error status before anything is enqueued.
+ *    A failed launch returns PA_ERR_CUDA.  pa_last_error_detail() gives a
+ *    human-readable reason for the last error on the calling thread.
+ *  - Checked mode: when `dev_error` is non-NULL (device memory, one int32
+ *    the caller zeroes), kernels validate device-resident indices and OR one
+ *    of the PA_DEVERR_* bits into it instead of reading or writing out of
+ *    range; the affected outputs are left unspecified.  Kernels never trap.
+ *    With dev_error == NULL the same checks run but nothing is reported:
+ *    cache accesses stay inside the cache either way (stores skip slots past
+ *    its end; reads go through TMA tensor maps, which zero-fill out-of-range
+ *    coordinates).
+ */
+#ifndef PAGED_KV_PA_H
+#define PAGED_KV_PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,   /* a pointer is NULL or misaligned, a size is negative, ...   */
+    PA_ERR_UNSUPPORTED = 2,   /* a valid shape this build has no kernel for                 */
+    PA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (launch, attribute, ...) */
+    PA_ERR_DEVICE_CHECK = 4,  /* a checked-mode kernel found a bad index (see PA_DEVERR_*)  */
+    PA_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out                         */
+    PA_ERR_WORKSPACE = 6      /* the workspace is NULL or smaller than the size query says  */
+} pa_status;
+
+/* Bits a kernel ORs into *dev_error in checked mode. */
+#define PA_DEVERR_BLOCK_ID    0x1  /* a block_table entry that a context needs is outside [0, num_blocks) */
+#define PA_DEVERR_SLOT        0x2  /* a slot_mapping entry is >= num_blocks * block_size                 */
+#define PA_DEVERR_CONTEXT_LEN 0x4  /* context_lens[s] < 1, > max_context_len or > table capacity         */
+#define PA_DEVERR_SEQLENS     0x8  /* cu_seqlens not monotone, n_new > n_k, or a length > max_seqlen     */
+#define PA_DEVERR_TIMEOUT     0x10 /* a bounded mbarrier wait gave up                                     */
+
+/* Static string naming a status code. */
+PA_API const char *pa_status_string(int status);
+
+/* Text describing the last error returned on the calling thread ("" if none). */
+PA_API const char *pa_last_error_detail(void);
+
+/* Library ABI version (major * 100 + minor). */
+PA_API int pa_version(void);
+
+/*
+ * pa_store_kv -- store_kvcache.
+ *
+ * For every i in [0, num_tokens) with slot_mapping[i] >= 0:
+ *     k_cache.view(num_blocks * block_size, num_kv_heads, head_dim)[slot_mapping[i]] = k[i]
+ *     v_cache.view(...)[slot_mapping[i]]                                          = v[i]
+ * a bit-exact copy ("a light kernel writes this step's K/V into the
+ * pre-allocated cache through slot_mapping", nano-vllm walkthrough, section
+ * seven; the Triton store kernel of the gitcode.csdn.net nano-vLLM article,
+ * section 3.4).  Negative slots are skipped (padding rows).  Two rows that
+ * name the same slot in one call race: the caller must not pass duplicates.
+ *
+ *   k, v           [num_tokens, num_kv_heads, head_dim] bf16; row i starts at
+ *                  element i * k_row_stride (resp. v_row_stride); each row's
+ *                  num_kv_heads * head_dim elements are contiguous.
+ *   slot_mapping   [num_tokens] int32, device.
+ *   k_cache/v_cache  the paged cache (written in place).
+ * num_tokens == 0 is a no-op that returns PA_OK.
+ */
+PA_API pa_status pa_store_kv(const void *k, const void *v, int64_t k_row_stride, int64_t v_row_stride,
+                      const int32_t *slot_mapping, int32_t num_tokens, void *k_cache, void *v_cache,
+                      int32_t num_blocks, int32_t block_size, int32_t num_kv_heads, int32_t head_dim,
+                      int32_t *dev_error, void *stream);
+
+/*
+ * Bytes of device workspace pa_decode needs for these sizes on the current
+ * device (0 when the decode runs in a single pass with no split).
+ */
+PA_API size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t block_size);
+
+/*
+ * pa_decode -- paged decode attention (the flash_attn_with_kvcache call with
+ * cache_seqlens = context_lens and block_table, nano-vllm walkthrough,
+ * section seven).  For every sequence s and q-head h:
+ *
+ *   out[s, h] = sum_j softmax_j(softmax_scale * q[s, h] . K_j) V_j,
+ *               j over the context_lens[s] tokens of sequence s,
+ *
+ * the attention formula of the chenxutan.com article (section 1.2), with K_j,
+ * V_j of KV head h / (num_q_heads / num_kv_heads) (GQA repeat_interleave,
+ * same article, section 3.2.1) gathered through block_table (the gather of the
+ * gsyq.cn article, sections 4.1 and 5.3).  context_lens counts the token
+ * stored by this step's pa_store_kv.
+ *
+ *   out, q           [batch, num_q_heads, head_dim] bf16, contiguous.
+ *   block_table      [batch, block_table_stride] int32; entries past
+ *                    ceil(context_lens[s] / block_size) are never read.
+ *   context_lens     [batch] int32, each in [1, max_context_len].
+ *   max_context_len  host-side upper bound of context_lens (sizes the split).
+ *   workspace        device scratch of at least pa_decode_workspace_size()
+ *                    bytes (may be NULL when that size is 0).  Its contents
+ *                    need no initialisation and are garbage afterwards.
+ *
+ * The work is split along each context (flash-decoding); per-split partial
+ * results in the workspace are merged by a second kernel on the same stream.
+ */
+PA_API pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_table, int32_t block_table_stride, const int32_t *context_lens,
+                    int32_t batch, int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads,
+                    int32_t head_dim, int32_t num_blocks, int32_t block_size, float softmax_scale,
+                    void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream);
+
+/*
+ * pa_decode_split -- pa_decode with the number of context splits chosen by
+ * the caller (num_splits > 0), like FlashAttention's num_splits argument;
+ * num_splits == 0 picks the split automatically, exactly as pa_decode does.
+ * The context is cut into splits of ceil(max_context_len / num_splits)
+ * tokens rounded up to a multiple of 64.  The result is the same function
+ * either way; only the rounding order of the fp32 accumulation changes.
+ * Workspace: pa_decode_split_workspace_size() with the same num_splits.
+ */
+PA_API size_t pa_decode_split_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                      int32_t max_context_len, int32_t num_splits);
+PA_API pa_status pa_decode_split(void *out, const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *block_table, int32_t block_table_stride, const int32_t *context_lens,
+                          int32_t batch, int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads,
+                          int32_t head_dim, int32_t num_blocks, int32_t block_size, float softmax_scale,
+                          int32_t num_splits, void *workspace, size_t workspace_bytes, int32_t *dev_error,
+                          void *stream);
+
+/* Bytes of device workspace pa_prefill_varlen needs (currently always 0). */
+PA_API size_t pa_prefill_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t num_q_heads,
+                                 int32_t num_kv_heads, int32_t head_dim);
+
+/*
+ * pa_prefill_varlen -- varlen causal prefill over the paged cache (the
+ * flash_attn_varlen_func call with cu_seqlens_q/k, max_seqlen_q/k,
+ * causal=True and block_table, nano-vllm walkthrough, section seven).
+ *
+ * Sequence s has n_new = cu_seqlens_q[s+1] - cu_seqlens_q[s] query tokens and
+ * n_k = cu_seqlens_k[s+1] - cu_seqlens_k[s] keys; the first c = n_k - n_new
+ * keys are a cached prefix (a prefix-cache hit) and the last n_new keys are
+ * the query tokens themselves, already stored by pa_store_kv.  New token i
+ * sits at absolute position c + i and, with causal != 0, attends to keys
+ * 0 .. c + i (all n_k keys when causal == 0):
+ *
+ *   out[cu_q[s] + i, h] = sum_j softmax_j(softmax_scale * q[cu_q[s] + i, h] . K_j) V_j
+ *
+ *   out, q           [total_q, num_q_heads, head_dim] bf16, contiguous,
+ *                    total_q = cu_seqlens_q[batch].
+ *   cu_seqlens_q/k   [batch + 1] int32, device, starting at 0.
+ *   max_seqlen_q/k   host-side upper bounds of n_new and n_k.
+ *   block_table      [batch, block_table_stride] int32.
+ */
+PA_API pa_status pa_prefill_varlen(void *out, const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t max_seqlen_q,
+                            int32_t max_seqlen_k, const int32_t *block_table, int32_t block_table_stride,
+                            int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                            int32_t num_blocks, int32_t block_size, float softmax_scale, int32_t causal,
+                            void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream);
+
+/*
+ * pa_selftest_bounded_wait -- exercises the library's bounded mbarrier wait:
+ * one CTA waits for an arrival that never comes, gives up after
+ * `max_polls` polls, ORs PA_DEVERR_TIMEOUT into *dev_error and exits
+ * normally, so the context stays usable.  Used by the tests of the timeout
+ * path; has no counterpart in the attention method itself.
+ */
+PA_API pa_status pa_selftest_bounded_wait(int32_t *dev_error, int64_t max_polls, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_KV_PA_H */

@@ -1,0 +1,403 @@
+// Paged GQA decode attention: split-KV flash-decoding plus a combine pass.
+//
+// What it computes (per sequence s, q-head h):
+//     out[s, h] = softmax_j(scale * q[s, h] . K_j) V_j  over the context of s,
+// the attention formula of the chenxutan.com Nano-vLLM article (section 1.2),
+// K_j / V_j taken from KV head h / G (GQA, same article, section 3.2.1) and
+// gathered through block_table (gsyq.cn article, sections 4.1 and 5.3) -- the
+// flash_attn_with_kvcache call of the nano-vllm walkthrough (section seven).
+//
+// How:
+//  * grid (split, kv_head, sequence); each CTA owns `chunk` consecutive tokens
+//    of one sequence's context for one KV head and ALL G q-heads of its GQA
+//    group, so every K/V byte is read from HBM once per call.
+//  * warp 4 is a TMA producer: for each 64-token tile it reads the tile's
+//    physical block ids from block_table and issues 3-D tensor-map loads
+//    (128-byte swizzle) of the K and V rows of this KV head into a 3-stage
+//    shared-memory ring guarded by mbarriers.
+//  * warps 0-3 each take 16 tokens of a tile: S = Q K^T and O += P V on the
+//    tensor cores with mma.sync m16n8k16 (bf16 in, fp32 accumulate), the G
+//    q-heads padded to the 16 rows of the A operand, online softmax in fp32
+//    (base-2 exponent, scale * log2(e) folded into the scores).
+//  * the four warps' (max, sum, O) are merged in shared memory; with one split
+//    the CTA writes bf16 out, otherwise a normalised fp32 partial and its
+//    log-sum-exp go to the workspace and decode_combine_kernel merges them.
+//  * masked positions (past the end of the context) are selected out: their
+//    score becomes -inf and their V rows are zeroed in registers, so stale or
+//    poisoned cache contents never reach the result (0 * NaN is never formed).
+#include <float.h>
+
+#include <atomic>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+constexpr int kTile = kDecodeTileTokens;  // tokens per pipeline stage
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kHalfBytes = kTile * 128;   // one 64-element slice of head_dim for 64 tokens
+
+template <int D>
+struct DecodeCfg {
+    static constexpr int kHalves = D / 64;
+    static constexpr int kStages = D == 128 ? 3 : 6;
+    static constexpr int kKvBytes = kHalves * kHalfBytes;        // K (or V) part of a stage
+    static constexpr int kStageBytes = 2 * kKvBytes;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kRedBytes = kConsumerWarps * 16 * (D + 2) * 4;
+    static_assert(kRedBytes <= kRingBytes, "reduction scratch must fit in the ring");
+    static constexpr int kSmemBytes = kRingBytes + 2 * kStages * 8 + 1024;  // + barriers + alignment slack
+};
+
+__device__ __forceinline__ void consumer_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        const DecodeArgs a) {
+    using C = DecodeCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kRingBytes);
+    uint64_t *empty = full + C::kStages;
+
+    const int split = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ctx = __ldg(a.context_lens + s);
+    if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size) {
+        if (split == 0 && kvh == 0 && threadIdx.x == 0) report(a.dev_error, PA_DEVERR_CONTEXT_LEN);
+        return;
+    }
+    const int t_begin = split * a.plan.chunk;
+    if (t_begin >= ctx) return;               // this split lies past the end of the context
+    const int t_end = min(ctx, t_begin + a.plan.chunk);
+    const int ntiles = (t_end - t_begin + kTile - 1) / kTile;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < C::kStages; ++st) {
+            mbar_init(smem_u32(full + st), 1);
+            mbar_init(smem_u32(empty + st), kConsumerWarps);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    const uint32_t ring = smem_u32(smem);
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------ producer --
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            const int32_t *bt = a.block_table + (int64_t)s * a.bt_stride;
+            const int B = a.block_size, box = a.box_tokens;
+            for (int i = 0; i < ntiles; ++i) {
+                const int st = i % C::kStages;
+                if (i >= C::kStages && !mbar_wait(smem_u32(empty + st), ((i / C::kStages) & 1) ^ 1, a.dev_error))
+                    break;
+                const int tile0 = t_begin + i * kTile;
+                const int nbox = (min(kTile, t_end - tile0) + box - 1) / box;
+                const uint32_t fb = smem_u32(full + st);
+                mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * 128 * C::kHalves * 2));
+                const uint32_t kdst = ring + st * C::kStageBytes;
+                const uint32_t vdst = kdst + C::kKvBytes;
+                for (int b = 0; b < nbox; ++b) {
+                    const int tok = tile0 + b * box;
+                    const int blk = __ldg(bt + tok / B);
+                    int row;
+                    if ((unsigned)blk < (unsigned)a.num_blocks) {
+                        row = blk * B + (tok % B);
+                    } else {               // out-of-range id: load zeros instead (TMA fills)
+                        report(a.dev_error, PA_DEVERR_BLOCK_ID);
+                        row = -box;
+                    }
+#pragma unroll
+                    for (int h = 0; h < C::kHalves; ++h) {
+                        const uint32_t off = h * kHalfBytes + b * box * 128;
+                        tma_load_3d(kdst + off, &tm_k, h * 64, kvh, row, fb);
+                        tma_load_3d(vdst + off, &tm_v, h * 64, kvh, row, fb);
+                    }
+                }
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers --
+    const int G = a.group;
+    const int g0 = lane >> 2;             // accumulator rows g0 and g0 + 8
+    const int c2 = (lane & 3) * 2;        // accumulator columns c2, c2 + 1
+    uint32_t qa[D / 16][4];
+    {
+        const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(a.q) +
+                                  ((int64_t)s * a.num_q_heads + (int64_t)kvh * G) * D;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const int k0 = ks * 16 + c2;
+            qa[ks][0] = g0 < G ? __ldg(reinterpret_cast<const uint32_t *>(qb + g0 * D + k0)) : 0u;
+            qa[ks][1] = g0 + 8 < G ? __ldg(reinterpret_cast<const uint32_t *>(qb + (g0 + 8) * D + k0)) : 0u;
+            qa[ks][2] = g0 < G ? __ldg(reinterpret_cast<const uint32_t *>(qb + g0 * D + k0 + 8)) : 0u;
+            qa[ks][3] = g0 + 8 < G ? __ldg(reinterpret_cast<const uint32_t *>(qb + (g0 + 8) * D + k0 + 8)) : 0u;
+        }
+    }
+
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+    float o[D / 8][4];
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+
+    const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: matrix index / row this lane addresses
+    bool ok = true;
+    for (int i = 0; i < ntiles; ++i) {
+        const int st = i % C::kStages;
+        const bool landed = mbar_wait(smem_u32(full + st), (i / C::kStages) & 1, a.dev_error);
+        if (!__all_sync(0xffffffffu, landed)) {   // leave together: the loop body uses full-warp shuffles
+            ok = false;
+            break;
+        }
+        const uint32_t kbase = ring + st * C::kStageBytes;
+        const uint32_t vbase = kbase + C::kKvBytes;
+        const int tok0 = t_begin + i * kTile + warp * 16;   // first token of this warp's slice
+
+        // S = Q K^T over this warp's 16 tokens (two n-tiles of 8 tokens)
+        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const int trow = warp * 16 + (mi >> 1) * 8 + mr;
+            const int dch = ks * 2 + (mi & 1);
+            uint32_t b0n0, b1n0, b0n1, b1n1;
+            ldmatrix_x4(kbase + (dch >> 3) * kHalfBytes + swz128(trow, dch & 7), b0n0, b1n0, b0n1, b1n1);
+            mma_bf16_16816(sc[0], qa[ks], b0n0, b1n0);
+            mma_bf16_16816(sc[1], qa[ks], b0n1, b1n1);
+        }
+
+        // scale into log2 units and select out positions past the end
+        const bool partial = tok0 + 16 > t_end;
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int tok = tok0 + n * 8 + c2 + (e & 1);
+                const float v = sc[n][e] * a.scale_log2;
+                sc[n][e] = (!partial || tok < t_end) ? v : -INFINITY;
+            }
+
+        // online softmax (rows g0 and g0 + 8)
+        float mx[2];
+        mx[0] = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+        mx[1] = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+        }
+        float corr[2], ref[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const float m_new = fmaxf(m_run[r], mx[r]);
+            ref[r] = m_new == -INFINITY ? 0.f : m_new;
+            corr[r] = fast_exp2(m_run[r] - ref[r]);
+            m_run[r] = m_new;
+        }
+        float p[2][4];
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) p[n][e] = fast_exp2(sc[n][e] - ref[e >> 1]);
+        l_run[0] = l_run[0] * corr[0] + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
+        l_run[1] = l_run[1] * corr[1] + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
+        if (!__all_sync(0xffffffffu, corr[0] == 1.f && corr[1] == 1.f)) {
+#pragma unroll
+            for (int nt = 0; nt < D / 8; ++nt) {
+                o[nt][0] *= corr[0];
+                o[nt][1] *= corr[0];
+                o[nt][2] *= corr[1];
+                o[nt][3] *= corr[1];
+            }
+        }
+        uint32_t pa[4];
+        pa[0] = pack_bf16(p[0][0], p[0][1]);
+        pa[1] = pack_bf16(p[0][2], p[0][3]);
+        pa[2] = pack_bf16(p[1][0], p[1][1]);
+        pa[3] = pack_bf16(p[1][2], p[1][3]);
+
+        // V fragments hold tokens tok0 + c2 + {0,1} (b0) and tok0 + 8 + c2 + {0,1} (b1)
+        uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
+        if (partial) {
+            vm0 = (tok0 + c2 < t_end ? 0x0000ffffu : 0u) | (tok0 + c2 + 1 < t_end ? 0xffff0000u : 0u);
+            vm1 = (tok0 + 8 + c2 < t_end ? 0x0000ffffu : 0u) | (tok0 + 9 + c2 < t_end ? 0xffff0000u : 0u);
+        }
+#pragma unroll
+        for (int jp = 0; jp < D / 16; ++jp) {
+            const int trow = warp * 16 + (mi & 1) * 8 + mr;
+            const int dch = jp * 2 + (mi >> 1);
+            uint32_t b0a, b1a, b0b, b1b;
+            ldmatrix_x4_trans(vbase + (dch >> 3) * kHalfBytes + swz128(trow, dch & 7), b0a, b1a, b0b, b1b);
+            b0a &= vm0;
+            b1a &= vm1;
+            b0b &= vm0;
+            b1b &= vm1;
+            mma_bf16_16816(o[2 * jp], pa, b0a, b1a);
+            mma_bf16_16816(o[2 * jp + 1], pa, b0b, b1b);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(empty + st));
+    }
+
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
+        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+    }
+
+    // ---------------------------------------------- merge the four warps --
+    consumer_sync();   // every consumer finished reading the ring
+    float *red_o = reinterpret_cast<float *>(smem);                       // [warp][16][D]
+    float *red_ml = red_o + kConsumerWarps * 16 * D;                      // [warp][16][2]
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int g = g0 + r * 8;
+        if (g < G) {
+            float *dst = red_o + (warp * 16 + g) * D;
+#pragma unroll
+            for (int nt = 0; nt < D / 8; ++nt) {
+                dst[nt * 8 + c2] = o[nt][2 * r];
+                dst[nt * 8 + c2 + 1] = o[nt][2 * r + 1];
+            }
+            if ((lane & 3) == 0) {
+                red_ml[(warp * 16 + g) * 2] = m_run[r];
+                red_ml[(warp * 16 + g) * 2 + 1] = l_run[r];
+            }
+        }
+    }
+    consumer_sync();
+    if (!ok) return;
+
+    const bool single = a.plan.max_splits == 1;
+    for (int e = threadIdx.x; e < G * D; e += kConsumerWarps * 32) {
+        const int g = e / D, d = e % D;
+        float mt = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) mt = fmaxf(mt, red_ml[(w * 16 + g) * 2]);
+        float lt = 0.f, ot = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+            const float mw = red_ml[(w * 16 + g) * 2];
+            const float f = mw == -INFINITY ? 0.f : fast_exp2(mw - mt);
+            lt += f * red_ml[(w * 16 + g) * 2 + 1];
+            ot += f * red_o[(w * 16 + g) * D + d];
+        }
+        const int h = kvh * G + g;
+        if (single) {
+            static_cast<__nv_bfloat16 *>(a.out)[((int64_t)s * a.num_q_heads + h) * D + d] = __float2bfloat16_rn(ot / lt);
+        } else {
+            const int64_t pi = ((int64_t)s * a.num_q_heads + h) * a.plan.max_splits + split;
+            a.part_o[pi * D + d] = ot / lt;
+            if (d == 0) a.part_lse[pi] = mt + __log2f(lt);
+        }
+    }
+}
+
+// Merge the per-split partials of one (sequence, q-head) by log-sum-exp.
+template <int D>
+__global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // partials of the split kernel are visible
+    const int h = blockIdx.x % a.num_q_heads;
+    const int s = blockIdx.x / a.num_q_heads;
+    const int ctx = __ldg(a.context_lens + s);
+    if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size) return;
+    const int nsplit = (ctx + a.plan.chunk - 1) / a.plan.chunk;
+    const int64_t base = ((int64_t)s * a.num_q_heads + h) * a.plan.max_splits;
+    float mt = -INFINITY;
+    for (int i = 0; i < nsplit; ++i) mt = fmaxf(mt, a.part_lse[base + i]);
+    float den = 0.f, num = 0.f;
+    const int d = threadIdx.x;
+    for (int i = 0; i < nsplit; ++i) {
+        const float w = fast_exp2(a.part_lse[base + i] - mt);
+        den += w;
+        num += w * a.part_o[(base + i) * D + d];
+    }
+    static_cast<__nv_bfloat16 *>(a.out)[((int64_t)s * a.num_q_heads + h) * D + d] = __float2bfloat16_rn(num / den);
+}
+
+template <int D>
+cudaError_t launch_decode_d(const DecodeArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                            cudaStream_t stream) {
+    using C = DecodeCfg<D>;
+    static std::atomic<uint64_t> configured{0};   // one bit per device whose attribute is set
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = uint64_t(1) << (dev & 63);
+    if (!(configured.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    const dim3 grid((unsigned)a.plan.max_splits, (unsigned)a.num_kv_heads, (unsigned)a.batch);
+    decode_split_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tm_k, tm_v, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || a.plan.max_splits == 1) return e;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.batch * a.num_q_heads));
+    cfg.blockDim = dim3(D);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, a);
+}
+
+}  // namespace
+
+DecodePlan plan_decode(int32_t batch, int32_t num_kv_heads, int32_t max_context_len, int32_t num_splits,
+                       int32_t num_sms) {
+    DecodePlan p;
+    const int64_t full = ((int64_t)max_context_len + kTile - 1) / kTile * kTile;
+    int64_t chunk;
+    if (num_splits > 0) {
+        chunk = ((int64_t)max_context_len + num_splits - 1) / num_splits;
+        chunk = (chunk + kTile - 1) / kTile * kTile;
+    } else {
+        // aim at about eight waves of two CTAs per SM over the whole batch, but
+        // never fewer than four tiles per CTA
+        const int64_t target = (int64_t)(num_sms > 0 ? num_sms : 148) * 2 * 8;
+        const int64_t pairs = (int64_t)batch * num_kv_heads;
+        chunk = ((int64_t)max_context_len * pairs + target - 1) / target;
+        chunk = (chunk + kTile - 1) / kTile * kTile;
+        if (chunk < 4 * kTile) chunk = 4 * kTile;
+    }
+    if (chunk > full) chunk = full;
+    if (chunk < kTile) chunk = kTile;
+    p.chunk = (int32_t)chunk;
+    p.max_splits = (int32_t)((max_context_len + chunk - 1) / chunk);
+    if (p.max_splits < 1) p.max_splits = 1;
+    return p;
+}
+
+size_t decode_workspace_bytes(const DecodePlan &plan, int32_t batch, int32_t num_q_heads, int32_t head_dim) {
+    if (plan.max_splits <= 1) return 0;
+    const size_t n = (size_t)batch * num_q_heads * plan.max_splits;
+    const size_t o_bytes = (n * head_dim * sizeof(float) + 255) / 256 * 256;
+    return o_bytes + n * sizeof(float);
+}
+
+cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                          cudaStream_t stream) {
+    if (a.head_dim == 128) return launch_decode_d<128>(a, tm_k, tm_v, stream);
+    return launch_decode_d<64>(a, tm_k, tm_v, stream);
+}
+
+}  // namespace pa

@@ -1,0 +1,333 @@
+// C-ABI front end of libpagedattn.so: host-side validation, TMA tensor-map
+// encoding and dispatch to the kernels.  Every entry point is declared and
+// documented in include/pa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <string>
+
+#include "pa.h"
+#include "pa_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+pa_status fail(pa_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+pa_status fail(pa_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+pa_status ok() {
+    g_last_error.clear();
+    return PA_OK;
+}
+
+pa_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(PA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool pow2(int32_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// cuTensorMapEncodeTiled from the driver, looked up at first use so that the
+// library loads (and its host-side checks run) on machines without a driver.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+int num_sms_current() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+// A [rows, heads, head_dim] bf16 tensor viewed in 3-D for TMA: dims (innermost
+// first) {head_dim, heads, rows}, box {64, box_heads, box_rows}, 128-byte
+// swizzle (each box row of 64 bf16 values is one 128-byte swizzle row).
+pa_status encode_rows(CUtensorMap *map, const void *base, int64_t rows, int32_t heads, int32_t head_dim,
+                      int32_t box_heads, int32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (no CUDA driver?)");
+    cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)heads, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)heads * head_dim * 2};
+    cuuint32_t box[3] = {64u, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return PA_OK;
+}
+
+pa_status check_cache_shape(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads, int32_t head_dim) {
+    if (num_blocks < 1 || num_kv_heads < 1) return fail(PA_ERR_INVALID_ARG, "num_blocks and num_kv_heads must be >= 1");
+    if (head_dim != 64 && head_dim != 128) return fail(PA_ERR_UNSUPPORTED, "head_dim %d not in {64, 128}", head_dim);
+    if (!pow2(block_size) || block_size < 16 || block_size > 256)
+        return fail(PA_ERR_UNSUPPORTED, "block_size %d is not a power of two in [16, 256]", block_size);
+    if ((int64_t)num_blocks * block_size >= (int64_t(1) << 31))
+        return fail(PA_ERR_UNSUPPORTED, "num_blocks * block_size must be < 2^31");
+    return PA_OK;
+}
+
+pa_status check_heads(int32_t num_q_heads, int32_t num_kv_heads) {
+    if (num_q_heads < 1 || num_kv_heads < 1) return fail(PA_ERR_INVALID_ARG, "head counts must be >= 1");
+    if (num_q_heads % num_kv_heads != 0)
+        return fail(PA_ERR_INVALID_ARG, "num_q_heads %d is not a multiple of num_kv_heads %d", num_q_heads,
+                    num_kv_heads);
+    if (num_q_heads / num_kv_heads > 16)
+        return fail(PA_ERR_UNSUPPORTED, "GQA group %d > 16", num_q_heads / num_kv_heads);
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *pa_status_string(int status) {
+    switch (status) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA";
+        case PA_ERR_DEVICE_CHECK: return "PA_ERR_DEVICE_CHECK";
+        case PA_ERR_TIMEOUT: return "PA_ERR_TIMEOUT";
+        case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+        default: return "PA_ERR_UNKNOWN";
+    }
+}
+
+const char *pa_last_error_detail(void) { return g_last_error.c_str(); }
+
+int pa_version(void) { return 100; }
+
+pa_status pa_store_kv(const void *k, const void *v, int64_t k_row_stride, int64_t v_row_stride,
+                      const int32_t *slot_mapping, int32_t num_tokens, void *k_cache, void *v_cache,
+                      int32_t num_blocks, int32_t block_size, int32_t num_kv_heads, int32_t head_dim,
+                      int32_t *dev_error, void *stream) {
+    if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "num_tokens < 0");
+    pa_status st = check_cache_shape(num_blocks, block_size, num_kv_heads, head_dim);
+    if (st != PA_OK) return st;
+    const int64_t row = (int64_t)num_kv_heads * head_dim;
+    if (k_row_stride < row || v_row_stride < row)
+        return fail(PA_ERR_INVALID_ARG, "row strides must be >= num_kv_heads * head_dim");
+    if (num_tokens == 0) return ok();
+    if (!k || !v || !slot_mapping || !k_cache || !v_cache) return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned(k, 2) || !aligned(v, 2) || !aligned(slot_mapping, 4) || !aligned(k_cache, 16) ||
+        !aligned(v_cache, 16) || (dev_error && !aligned(dev_error, 4)))
+        return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
+    pa::StoreArgs a;
+    a.k = k;
+    a.v = v;
+    a.k_row_stride = k_row_stride;
+    a.v_row_stride = v_row_stride;
+    a.slot_mapping = slot_mapping;
+    a.num_tokens = num_tokens;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.num_slots = (int64_t)num_blocks * block_size;
+    a.row_elems = (int32_t)row;
+    a.dev_error = dev_error;
+    cudaError_t e = pa::launch_store(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "store kernel launch");
+    return ok();
+}
+
+size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t block_size) {
+    (void)block_size;
+    if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
+    pa::DecodePlan plan = pa::plan_decode(batch, num_kv_heads, max_context_len, 0, num_sms_current());
+    return pa::decode_workspace_bytes(plan, batch, num_q_heads, head_dim);
+}
+
+static pa_status decode_impl(void *out, const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *block_table, int32_t block_table_stride, const int32_t *context_lens,
+                             int32_t batch, int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads,
+                             int32_t head_dim, int32_t num_blocks, int32_t block_size, float softmax_scale,
+                             int32_t num_splits, void *workspace, size_t workspace_bytes, int32_t *dev_error,
+                             void *stream) {
+    if (batch < 0) return fail(PA_ERR_INVALID_ARG, "batch < 0");
+    pa_status st = check_cache_shape(num_blocks, block_size, num_kv_heads, head_dim);
+    if (st != PA_OK) return st;
+    if ((st = check_heads(num_q_heads, num_kv_heads)) != PA_OK) return st;
+    if (!(softmax_scale > 0.f) || !isfinite(softmax_scale))
+        return fail(PA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if (batch == 0) return ok();
+    if (max_context_len < 1) return fail(PA_ERR_INVALID_ARG, "max_context_len must be >= 1");
+    if (block_table_stride < 1) return fail(PA_ERR_INVALID_ARG, "block_table_stride must be >= 1");
+    if (num_splits < 0) return fail(PA_ERR_INVALID_ARG, "num_splits < 0");
+    if (!out || !q || !k_cache || !v_cache || !block_table || !context_lens)
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_table, 4) || !aligned(context_lens, 4) || (dev_error && !aligned(dev_error, 4)))
+        return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
+
+    pa::DecodeArgs a;
+    a.plan = pa::plan_decode(batch, num_kv_heads, max_context_len, num_splits, num_sms_current());
+    const size_t need = pa::decode_workspace_bytes(a.plan, batch, num_q_heads, head_dim);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need)
+            return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                        workspace ? workspace_bytes : (size_t)0);
+        if (!aligned(workspace, 256)) return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    }
+    a.out = out;
+    a.q = q;
+    a.block_table = block_table;
+    a.context_lens = context_lens;
+    a.dev_error = dev_error;
+    const size_t n = (size_t)batch * num_q_heads * a.plan.max_splits;
+    a.part_o = static_cast<float *>(workspace);
+    a.part_lse = need ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                  (n * head_dim * sizeof(float) + 255) / 256 * 256)
+                      : nullptr;
+    a.bt_stride = block_table_stride;
+    a.batch = batch;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.group = num_q_heads / num_kv_heads;
+    a.head_dim = head_dim;
+    a.num_blocks = num_blocks;
+    a.block_size = block_size;
+    a.box_tokens = block_size < pa::kDecodeTileTokens ? block_size : pa::kDecodeTileTokens;
+    a.max_context_len = max_context_len;
+    a.scale_log2 = softmax_scale * 1.4426950408889634f;
+
+    CUtensorMap tm_k, tm_v;
+    const int64_t rows = (int64_t)num_blocks * block_size;
+    if ((st = encode_rows(&tm_k, k_cache, rows, num_kv_heads, head_dim, 1, a.box_tokens)) != PA_OK) return st;
+    if ((st = encode_rows(&tm_v, v_cache, rows, num_kv_heads, head_dim, 1, a.box_tokens)) != PA_OK) return st;
+    cudaError_t e = pa::launch_decode(a, tm_k, tm_v, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+    return ok();
+}
+
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+                    int32_t block_table_stride, const int32_t *context_lens, int32_t batch, int32_t max_context_len,
+                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                    int32_t block_size, float softmax_scale, void *workspace, size_t workspace_bytes,
+                    int32_t *dev_error, void *stream) {
+    return decode_impl(out, q, k_cache, v_cache, block_table, block_table_stride, context_lens, batch,
+                       max_context_len, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, softmax_scale,
+                       0, workspace, workspace_bytes, dev_error, stream);
+}
+
+size_t pa_decode_split_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                      int32_t max_context_len, int32_t num_splits) {
+    if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_context_len <= 0 ||
+        num_splits < 0)
+        return 0;
+    pa::DecodePlan plan = pa::plan_decode(batch, num_kv_heads, max_context_len, num_splits, num_sms_current());
+    return pa::decode_workspace_bytes(plan, batch, num_q_heads, head_dim);
+}
+
+pa_status pa_decode_split(void *out, const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *block_table, int32_t block_table_stride, const int32_t *context_lens,
+                          int32_t batch, int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads,
+                          int32_t head_dim, int32_t num_blocks, int32_t block_size, float softmax_scale,
+                          int32_t num_splits, void *workspace, size_t workspace_bytes, int32_t *dev_error,
+                          void *stream) {
+    return decode_impl(out, q, k_cache, v_cache, block_table, block_table_stride, context_lens, batch,
+                       max_context_len, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, softmax_scale,
+                       num_splits, workspace, workspace_bytes, dev_error, stream);
+}
+
+size_t pa_prefill_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t head_dim) {
+    (void)batch, (void)max_seqlen_q, (void)num_q_heads, (void)num_kv_heads, (void)head_dim;
+    return 0;
+}
+
+pa_status pa_prefill_varlen(void *out, const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t max_seqlen_q,
+                            int32_t max_seqlen_k, const int32_t *block_table, int32_t block_table_stride,
+                            int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                            int32_t num_blocks, int32_t block_size, float softmax_scale, int32_t causal,
+                            void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream) {
+    (void)workspace, (void)workspace_bytes;
+    if (batch < 0) return fail(PA_ERR_INVALID_ARG, "batch < 0");
+    pa_status st = check_cache_shape(num_blocks, block_size, num_kv_heads, head_dim);
+    if (st != PA_OK) return st;
+    if ((st = check_heads(num_q_heads, num_kv_heads)) != PA_OK) return st;
+    if (128 % (num_q_heads / num_kv_heads) != 0)
+        return fail(PA_ERR_UNSUPPORTED, "prefill needs a GQA group that divides 128");
+    if (!(softmax_scale > 0.f) || !isfinite(softmax_scale))
+        return fail(PA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if (batch == 0 || max_seqlen_q == 0) return ok();
+    if (max_seqlen_q < 0 || max_seqlen_k < 1 || max_seqlen_k < max_seqlen_q)
+        return fail(PA_ERR_INVALID_ARG, "need 0 <= max_seqlen_q <= max_seqlen_k and max_seqlen_k >= 1");
+    if (block_table_stride < 1) return fail(PA_ERR_INVALID_ARG, "block_table_stride must be >= 1");
+    if (!out || !q || !k_cache || !v_cache || !cu_seqlens_q || !cu_seqlens_k || !block_table)
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) || !aligned(block_table, 4) ||
+        (dev_error && !aligned(dev_error, 4)))
+        return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
+
+    pa::PrefillArgs a;
+    a.out = out;
+    a.q = q;
+    a.cu_q = cu_seqlens_q;
+    a.cu_k = cu_seqlens_k;
+    a.block_table = block_table;
+    a.dev_error = dev_error;
+    a.bt_stride = block_table_stride;
+    a.batch = batch;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.group = num_q_heads / num_kv_heads;
+    a.head_dim = head_dim;
+    a.num_blocks = num_blocks;
+    a.block_size = block_size;
+    a.box_tokens = block_size < 128 ? block_size : 128;
+    a.max_seqlen_q = max_seqlen_q;
+    a.max_seqlen_k = max_seqlen_k;
+    a.causal = causal ? 1 : 0;
+    a.scale_log2 = softmax_scale * 1.4426950408889634f;
+
+    CUtensorMap tm_k, tm_v;
+    const int64_t rows = (int64_t)num_blocks * block_size;
+    if ((st = encode_rows(&tm_k, k_cache, rows, num_kv_heads, head_dim, 1, a.box_tokens)) != PA_OK) return st;
+    if ((st = encode_rows(&tm_v, v_cache, rows, num_kv_heads, head_dim, 1, a.box_tokens)) != PA_OK) return st;
+    cudaError_t e = pa::launch_prefill(a, tm_k, tm_v, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return fail(PA_ERR_UNSUPPORTED, "prefill kernel not available");
+    if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
+    return ok();
+}
+
+pa_status pa_selftest_bounded_wait(int32_t *dev_error, int64_t max_polls, void *stream) {
+    if (!dev_error || !aligned(dev_error, 4)) return fail(PA_ERR_INVALID_ARG, "dev_error must be a device int32");
+    if (max_polls < 1 || max_polls > (int64_t(1) << 30)) return fail(PA_ERR_INVALID_ARG, "max_polls out of range");
+    cudaError_t e = pa::launch_selftest_wait(dev_error, max_polls, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// Internal interfaces between the C-ABI front end (pa_api.cu) and the kernel
+// translation units.  Not installed; not part of the ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+// ----------------------------------------------------------------- store --
+struct StoreArgs {
+    const void *k, *v;
+    int64_t k_row_stride, v_row_stride;   // elements
+    const int32_t *slot_mapping;
+    int32_t num_tokens;
+    void *k_cache, *v_cache;
+    int64_t num_slots;
+    int32_t row_elems;                    // num_kv_heads * head_dim
+    int32_t *dev_error;
+};
+cudaError_t launch_store(const StoreArgs &a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- decode --
+constexpr int kDecodeTileTokens = 64;
+
+struct DecodePlan {
+    int32_t chunk;       // tokens per split, a multiple of kDecodeTileTokens
+    int32_t max_splits;  // splits of the longest context
+};
+DecodePlan plan_decode(int32_t batch, int32_t num_kv_heads, int32_t max_context_len, int32_t num_splits,
+                       int32_t num_sms);
+size_t decode_workspace_bytes(const DecodePlan &plan, int32_t batch, int32_t num_q_heads, int32_t head_dim);
+
+struct DecodeArgs {
+    void *out;
+    const void *q;
+    const int32_t *block_table;
+    const int32_t *context_lens;
+    int32_t *dev_error;
+    float *part_o;      // [batch, Hq, max_splits, D]
+    float *part_lse;    // [batch, Hq, max_splits]
+    int32_t bt_stride, batch, num_q_heads, num_kv_heads, group, head_dim;
+    int32_t num_blocks, block_size, box_tokens, max_context_len;
+    DecodePlan plan;
+    float scale_log2;
+};
+cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                          cudaStream_t stream);
+
+// --------------------------------------------------------------- prefill --
+struct PrefillArgs {
+    void *out;
+    const void *q;
+    const int32_t *cu_q, *cu_k, *block_table;
+    int32_t *dev_error;
+    int32_t bt_stride, batch, num_q_heads, num_kv_heads, group, head_dim;
+    int32_t num_blocks, block_size, box_tokens, max_seqlen_q, max_seqlen_k, causal;
+    float scale_log2;
+};
+cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                           cudaStream_t stream);
+
+// ------------------------------------------------------------- self-test --
+cudaError_t launch_selftest_wait(int32_t *dev_error, int64_t max_polls, cudaStream_t stream);
+
+}  // namespace pa

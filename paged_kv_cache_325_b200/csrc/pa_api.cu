@@ -284,6 +284,8 @@ pa_status pa_prefill_varlen(void *out, const void *q, const void *k_cache, const
     if (max_seqlen_q < 0 || max_seqlen_k < 1 || max_seqlen_k < max_seqlen_q)
         return fail(PA_ERR_INVALID_ARG, "need 0 <= max_seqlen_q <= max_seqlen_k and max_seqlen_k >= 1");
     if (block_table_stride < 1) return fail(PA_ERR_INVALID_ARG, "block_table_stride must be >= 1");
+    if ((int64_t)max_seqlen_q > (int64_t)65535 * (128 / (num_q_heads / num_kv_heads)))
+        return fail(PA_ERR_UNSUPPORTED, "max_seqlen_q %d is too long for one launch", max_seqlen_q);
     if (!out || !q || !k_cache || !v_cache || !cu_seqlens_q || !cu_seqlens_k || !block_table)
         return fail(PA_ERR_INVALID_ARG, "NULL pointer");
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||

@@ -14,11 +14,9 @@
 
 namespace pa {
 
-// Poll budget of every bounded wait (each poll is a try_wait, which itself
-// suspends for a hardware-defined interval, plus a short nanosleep after the
-// first few polls).  At roughly 0.1-1 us per poll this gives up after about
-// one to ten seconds, far beyond any legitimate wait in these kernels.
-constexpr uint32_t kWaitPolls = 1u << 24;
+// Every bounded wait gives up after this much wall-clock time (read from the
+// %globaltimer nanosecond clock), far beyond any legitimate wait here.
+constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
 
 PA_DEVICE uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -64,12 +62,21 @@ PA_DEVICE bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+PA_DEVICE uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false (and
-// reports PA_DEVERR_TIMEOUT) if it did not complete within `polls` polls.
-PA_DEVICE bool mbar_wait(uint32_t bar, uint32_t parity, int32_t *dev_error, uint32_t polls = kWaitPolls) {
-    for (uint32_t i = 0; i < polls; ++i) {
+// reports PA_DEVERR_TIMEOUT) if it did not complete within kWaitTimeoutNs or
+// within `max_polls` polls, whichever comes first.
+PA_DEVICE bool mbar_wait(uint32_t bar, uint32_t parity, int32_t *dev_error, uint32_t max_polls = 0xffffffffu) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1; i < max_polls; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (i >= 32) __nanosleep(64);
+        if ((i & 63u) == 0 && global_timer_ns() - t0 > kWaitTimeoutNs) break;
     }
     report(dev_error, PA_DEVERR_TIMEOUT);
     return false;

@@ -1,0 +1,521 @@
+#!/usr/bin/env python
+"""Benchmark of the paged-KV hot path on B200: store_kvcache + paged decode
+(+ varlen prefill), through the C ABI of libpagedattn.so.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+One step = one attention-layer call of the Qwen3-0.6B-like decode workload
+(batch 64, context lengths U[100, 1024], 16 q / 8 kv heads, head_dim 128,
+block_size 256): pa_store_kv of the 64 new K/V rows, then pa_decode (split
+kernel + combine).  `value` is decode tokens/s over all ranks (each rank runs
+its own replica: the path shards by sequence with no exchange, so scaling is
+weak).  Inputs are resident in HBM; L2 is flushed (256 MiB write) before
+every timed step; each step is timed with CUDA events on the launching
+stream.  The same line carries the long-context, prefix-sharing and varlen
+prefill workloads (at N=1), the roofline of the dominant kernel, an end-to-end
+figure through the C ABI with host buffers, the CPU oracle baseline and the
+SM clocks sampled during the timed region.
+
+For N > 1 launch with torch.distributed.run (one rank per GPU, NCCL); rank 0
+prints the single JSON line.  ``--impl reference`` times the CPU oracle (the
+reference arm): rank 0 only, a bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode tokens/s and KV HBM GB/s (% of B200 peak); prefill TFLOP/s"
+PRIMARY = "qwen3_0.6b_decode"
+PRIMARY_DESC = ("Qwen3-0.6B-like decode layer call: batch 64, context_lens U[100,1024], 16 q / 8 kv heads, "
+                "head_dim 128, block_size 256, shuffled blocks; pa_store_kv of 64 new rows + pa_decode")
+FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers --
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(relpath):
+    with open(os.path.join(ROOT, relpath), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch recorded from an ncu capture (profiles/traffic.txt), or None
+    when the kernel source changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        m = re.match(r"\s*(\S+)\s+source=(\S+)\s+sha=(\w+)\s+bytes_per_launch=(\d+)", line)
+        if m and m.group(1) == kernel and source_sha(m.group(2)) == m.group(3):
+            return int(m.group(4))
+    return None
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 6:
+                continue
+            try:
+                mhz.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[2:]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}: launch N>1 with torch.distributed.run")
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Maximum of a per-rank float over all ranks (the only collective, outside timing)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def aggregate(local_time_s: float, local_units: float, world: int, device):
+    """Whole-job throughput: units of all ranks / the slowest rank's time."""
+    t = max_over_ranks(local_time_s, world, device)
+    u = sum_over_ranks(local_units, world, device)
+    return u / t, t
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------- native timing --
+
+class Timer:
+    """Per-step CUDA events on the current (launching) stream, L2 flushed between steps."""
+
+    def __init__(self, device):
+        self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def run(self, parts, steps, flush=True):
+        """parts: list of callables run in order each step; returns per-part lists of seconds."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)] for _ in range(steps)]
+        for i in range(steps):
+            if flush:
+                self.flush.zero_()
+            ev[i][0].record()
+            for j, p in enumerate(parts):
+                p()
+                ev[i][j + 1].record()
+        torch.cuda.synchronize()
+        return [[ev[i][j].elapsed_time(ev[i][j + 1]) * 1e-3 for i in range(steps)] for j in range(len(parts))]
+
+
+def capture(fn):
+    """Capture fn into a CUDA graph (after one eager call); returns graph.replay."""
+    fn()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g.replay, g
+
+
+class DecodeBench:
+    def __init__(self, case, device):
+        import paged_kv_cache_325_b200 as pa
+        from paged_kv_cache_325_b200.workloads import DecodeCase  # noqa: F401
+        self.pa = pa
+        self.case = case
+        self.dev = device
+        c = case
+        self.k_cache = c.k_cache.to(device)
+        self.v_cache = c.v_cache.to(device)
+        self.k_new = c.k_new.to(device)
+        self.v_new = c.v_new.to(device)
+        self.q = c.q.to(device)
+        self.slot = torch.as_tensor(c.slot_mapping).to(device)
+        self.bt = torch.as_tensor(c.block_table).to(device)
+        self.ctx = torch.as_tensor(c.context_lens).to(device)
+        self.out = torch.empty_like(self.q)
+        self.mcl = c.max_context_len
+        self.ws = pa.alloc_decode_workspace(self.q, c.num_kv_heads, self.mcl, c.block_size)
+        self.splits = self.ws.numel() > 1
+
+    def store(self):
+        self.pa.pa_store_kv(self.k_new, self.v_new, self.slot, self.k_cache, self.v_cache)
+
+    def decode(self):
+        c = self.case
+        self.pa.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.bt, self.ctx, self.mcl, c.softmax_scale,
+                          workspace=self.ws)
+
+    def launches_per_step(self):
+        return 1 + 1 + (1 if self.splits else 0)
+
+    def alg_bytes_decode(self):
+        c = self.case
+        return c.kv_bytes_read() + 2 * self.q.numel() * 2 + c.batch * 4 + self.bt.numel() * 4
+
+    def alg_bytes_store(self):
+        return 2 * 2 * self.k_new.numel() * 2 + self.slot.numel() * 4
+
+
+def bench_primary(args, world, rank, device, pk):
+    from paged_kv_cache_325_b200 import workloads as W
+    case = W.WORKLOADS[PRIMARY](poison=False, keep_contiguous=False)
+    b = DecodeBench(case, device)
+    st_replay, _g1 = capture(b.store)
+    dec_replay, _g2 = capture(b.decode)
+    timer = Timer(device)
+    timer.run([st_replay, dec_replay], max(args.warmup, 3))
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local_gpu_index(device)) as clk:
+        t_store, t_dec = timer.run([st_replay, dec_replay], args.steps)
+    torch.cuda.synchronize()
+    barrier(world)
+    local_total = sum(t_store) + sum(t_dec)
+    value, t_max = aggregate(local_total, args.steps * case.batch, world, device)
+    dec_mean = statistics.mean(t_dec)
+    achieved = b.alg_bytes_decode() / dec_mean / 1e9
+    res = {
+        "value": value, "ms_per_step": t_max / args.steps * 1e3,
+        "kv_gbps": case.kv_bytes_read() / dec_mean / 1e9,
+        "kv_hbm_frac_of_measured": case.kv_bytes_read() / dec_mean / 1e9 / pk["hbm_gbs"],
+        "kv_hbm_frac_of_8tbs": case.kv_bytes_read() / dec_mean / 1e9 / 8000.0,
+        "store_us": statistics.mean(t_store) * 1e6, "decode_us": dec_mean * 1e6,
+        "roofline": {"kernel": "decode_split_kernel<128> + decode_combine_kernel", "bound": "hbm",
+                     "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                     "traffic": recorded_traffic("decode_qwen3_0.6b"),
+                     "alg_bytes_per_launch": b.alg_bytes_decode()},
+        "gpu_launches": b.launches_per_step() * args.steps,
+        "clocks": clk.summary(),
+    }
+    res["e2e"] = bench_e2e(b, args, world, device)
+    return case, res
+
+
+def bench_e2e(b, args, world, device):
+    """Same metric through the public API with pinned host buffers: per step, H2D of the step's
+    inputs, store + decode, D2H of the output, all inside the timed region."""
+    host = {}
+    for name in ("q", "k_new", "v_new", "slot", "bt", "ctx"):
+        t = getattr(b, name)
+        host[name] = t.detach().cpu().pin_memory()
+    out_h = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def step():
+        for name, t in host.items():
+            getattr(b, name).copy_(t, non_blocking=True)
+        b.store()
+        b.decode()
+        out_h.copy_(b.out, non_blocking=True)
+
+    timer = Timer(device)
+    timer.run([step], max(args.warmup, 3))
+    steps = max(1, min(args.steps, 500))
+    barrier(world)
+    (ts,) = timer.run([step], steps)
+    barrier(world)
+    value, _ = aggregate(sum(ts), steps * b.case.batch, world, device)
+    return {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": steps}
+
+
+def bench_secondary(args, device, pk, names):
+    """Long-context and prefix-sharing decode, varlen prefill: rank 0 at N=1."""
+    import paged_kv_cache_325_b200 as pa
+    from paged_kv_cache_325_b200 import workloads as W
+    timer = Timer(device)
+    out = {}
+    steps = max(10, min(args.steps, 200))
+    for name in [n for n in names if n in ("long_context_decode", "prefix_sharing_decode")]:
+        case = W.WORKLOADS[name](poison=False, keep_contiguous=False)
+        b = DecodeBench(case, device)
+        b.store()
+        dec_replay, _g = capture(b.decode)
+        timer.run([dec_replay], 5)
+        (t,) = timer.run([dec_replay], steps)
+        tm = statistics.mean(t)
+        ach = b.alg_bytes_decode() / tm / 1e9
+        r = {"decode_us": tm * 1e6, "tokens_per_s": case.batch / tm,
+             "kv_gbps_logical": case.kv_bytes_read() / tm / 1e9,
+             "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                          "frac": ach / pk["hbm_gbs"], "frac_of_8tbs": ach / 8000.0}}
+        if name == "prefix_sharing_decode":
+            uniq = case.kv_bytes_unique() + 2 * b.q.numel() * 2
+            r["kv_gbps_unique"] = case.kv_bytes_unique() / tm / 1e9
+            r["roofline"] = {"bound": "hbm", "achieved": uniq / tm / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": uniq / tm / 1e9 / pk["hbm_gbs"], "bytes": "unique"}
+            (tw,) = timer.run([dec_replay], steps, flush=False)
+            r["decode_us_warm_l2"] = statistics.mean(tw) * 1e6
+        out[name] = r
+        del b, dec_replay, _g
+        torch.cuda.empty_cache()
+    if "varlen_prefill" not in names:
+        return out
+    case = W.varlen_prefill(poison=False, keep_contiguous=False)
+    dev = device
+    kc, vc = case.k_cache.to(dev), case.v_cache.to(dev)
+    kn, vn, q = case.k_new.to(dev), case.v_new.to(dev), case.q.to(dev)
+    slot = torch.as_tensor(case.slot_mapping).to(dev)
+    bt = torch.as_tensor(case.block_table).to(dev)
+    cq = torch.as_tensor(case.cu_seqlens_q).to(dev)
+    ck = torch.as_tensor(case.cu_seqlens_k).to(dev)
+    o = torch.empty_like(q)
+
+    def st():
+        pa.pa_store_kv(kn, vn, slot, kc, vc)
+
+    def pf():
+        pa.pa_prefill_varlen(o, q, kc, vc, cq, ck, case.max_seqlen_q, case.max_seqlen_k, bt, case.softmax_scale)
+
+    st_replay, _g1 = capture(st)
+    pf_replay, _g2 = capture(pf)
+    timer.run([st_replay, pf_replay], 5)
+    ts, tp = timer.run([st_replay, pf_replay], steps)
+    tpm, tsm = statistics.mean(tp), statistics.mean(ts)
+    fl = case.causal_flops()
+    ach = fl / tpm / 1e12
+    store_bytes = 2 * 2 * kn.numel() * 2
+    out["varlen_prefill"] = {
+        "prefill_us": tpm * 1e6, "store_us": tsm * 1e6, "causal_tflop": fl / 1e12,
+        "tflops": ach, "new_tokens": case.total_q, "prefill_tokens_per_s": case.total_q / (tpm + tsm),
+        "store_gbps": store_bytes / tsm / 1e9,
+        "roofline": {"kernel": "prefill_kernel<128>", "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
+                     "frac_of_sustained": ach / pk["bf16_tflops_sustained"],
+                     "traffic": recorded_traffic("prefill_varlen")},
+    }
+    return out
+
+
+def local_gpu_index(device):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    idx = device.index or 0
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if idx < len(ids) and ids[idx].isdigit():
+            return int(ids[idx])
+    return idx
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def oracle_decode_sample(case, n_seq, rng):
+    """Oracle store + decode of n_seq randomly chosen sequences (all q-heads); returns seconds."""
+    import oracle
+    seqs = rng.choice(case.batch, size=n_seq, replace=False)
+    t0 = time.perf_counter()
+    oracle.store(case.k_new, case.v_new, case.slot_mapping, case.k_cache, case.v_cache)
+    si = np.repeat(seqs, case.num_q_heads)
+    hi = np.tile(np.arange(case.num_q_heads), n_seq)
+    oracle.decode(case.q, case.k_cache, case.v_cache, case.block_table, case.context_lens, case.softmax_scale,
+                  seq_idx=si, head_idx=hi)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(case, budget_s=10.0):
+    import oracle
+    rng = np.random.default_rng(0)
+    t1 = oracle_decode_sample(case, 8, rng)
+    reps, total, toks = 0, 0.0, 0
+    while total < budget_s and reps < 1000:
+        total += oracle_decode_sample(case, 8, rng)
+        toks += 8
+        reps += 1
+    return {"value": toks / total, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{reps} x (oracle store of all 64 rows + fp64 decode of 8 random sequences x 16 heads) "
+                      f"of the {PRIMARY} workload, {total:.1f} s; first call {t1:.2f} s excluded"}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle as it stands, a bounded sample per step (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    from paged_kv_cache_325_b200 import workloads as W
+    case = W.WORKLOADS[PRIMARY](poison=False, keep_contiguous=False)
+    rng = np.random.default_rng(0)
+    t1 = oracle_decode_sample(case, 1, rng)
+    per_step_budget = 90.0 / max(1, args.steps + args.warmup)
+    n_seq = int(max(1, min(case.batch, per_step_budget / max(t1, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_decode_sample(case, n_seq, rng)
+    ts = [oracle_decode_sample(case, n_seq, rng) for _ in range(args.steps)]
+    value = n_seq * args.steps / sum(ts)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(ts) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": PRIMARY_DESC, "parallelism": "replicas", "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"per step: oracle store of 64 rows + fp64 decode of {n_seq} random "
+                                       f"sequences x 16 heads of the {PRIMARY} workload"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main --
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--secondary", default="long_context_decode,prefix_sharing_decode,varlen_prefill",
+                    help="comma list of extra workloads to time at N=1 ('none' for none)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return 0
+
+    import paged_kv_cache_325_b200 as pa
+    pa.load_library()            # fails loudly when the CUDA library is missing
+    if not torch.cuda.is_available():
+        raise SystemExit("no CUDA device: the native arm has no CPU path")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    pk, peak_src = peaks()
+    try:
+        case, res = bench_primary(args, world, rank, device, pk)
+        secondary = None
+        names = [n for n in args.secondary.split(",") if n and n != "none"]
+        if world == 1 and names:
+            secondary = bench_secondary(args, device, pk, names)
+        cpu = None
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(case)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    rf = res["roofline"]
+    rf["peak_source"] = peak_src
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": PRIMARY_DESC, "parallelism": f"replicas x{world}",
+                   "l2": "flushed between timed steps (256 MiB write)",
+                   "timing": "per-step CUDA events around CUDA-graph replays of store and decode"},
+        "kv_gbps": res["kv_gbps"], "kv_hbm_frac_of_measured": res["kv_hbm_frac_of_measured"],
+        "kv_hbm_frac_of_8tbs": res["kv_hbm_frac_of_8tbs"], "store_us": res["store_us"],
+        "decode_us": res["decode_us"], "roofline": rf, "cpu_baseline": cpu, "e2e": res["e2e"],
+        "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
+    }
+    if secondary is not None:
+        line["workloads"] = secondary
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

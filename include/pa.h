@@ -170,6 +170,35 @@ PA_API pa_status pa_decode_split(void *out, const void *q, const void *k_cache, 
                           int32_t num_splits, void *workspace, size_t workspace_bytes, int32_t *dev_error,
                           void *stream);
 
+/*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
+ * memory (no counterpart in the pages: it exists for integration, not for the
+ * method).  Some hosts own every device allocation themselves -- a plugin
+ * runtime, or an engine that gives all spare HBM to its KV-cache pool -- and
+ * cannot hand this library a workspace.  This variant computes exactly what
+ * pa_decode computes, but takes its split scratch from a fixed array compiled
+ * into the library: pa_decode_noalloc_max_scratch_bytes() bytes (8 MiB) per
+ * GPU, held by every GPU that loads the library until the process exits.  It
+ * calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments are those of pa_decode without the workspace.  Sizes whose split
+ * scratch (pa_decode_workspace_size) exceeds the array are rejected with
+ * PA_ERR_WORKSPACE before anything is enqueued.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress, that device
+ * current) and caches it; make that first call before any stream capture.
+ * Every call on a device shares the one array and it keeps the last call's
+ * contents; nothing in it has to start at zero (each call writes every
+ * partial it reads).  Calls whose kernels overlap on the GPU -- on different
+ * streams, or concurrently from several host threads -- race on the array:
+ * serialise them (one stream, or events).
+ */
+PA_API size_t pa_decode_noalloc_max_scratch_bytes(void);
+PA_API pa_status pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                   const int32_t *block_table, int32_t block_table_stride,
+                                   const int32_t *context_lens, int32_t batch, int32_t max_context_len,
+                                   int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                                   int32_t block_size, float softmax_scale, int32_t *dev_error, void *stream);
+
 /* Bytes of device workspace pa_prefill_varlen needs (currently always 0). */
 PA_API size_t pa_prefill_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t num_q_heads,
                                  int32_t num_kv_heads, int32_t head_dim);

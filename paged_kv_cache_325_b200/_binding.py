@@ -33,7 +33,7 @@ PA_DEVERR_SEQLENS = 0x8
 PA_DEVERR_TIMEOUT = 0x10
 
 __all__ = ["PagedAttnError", "load_library", "declared_symbols", "pa_store_kv", "pa_decode", "pa_decode_split",
-           "pa_decode_workspace_size", "pa_decode_split_workspace_size", "pa_prefill_varlen",
+           "pa_decode_workspace_size", "pa_decode_split_workspace_size", "pa_decode_noalloc", "pa_prefill_varlen",
            "pa_prefill_workspace_size", "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
            "alloc_decode_workspace"]
 
@@ -58,6 +58,9 @@ _SIGS = {
                                  _c_i32, _c_i32, _c_i32, _c_f32, _c_p, _c_sz, _c_p, _c_p]),
     "pa_decode_split": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_i32,
                                        _c_i32, _c_i32, _c_i32, _c_f32, _c_i32, _c_p, _c_sz, _c_p, _c_p]),
+    "pa_decode_noalloc_max_scratch_bytes": (_c_sz, []),
+    "pa_decode_noalloc": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_i32,
+                                         _c_i32, _c_i32, _c_i32, _c_f32, _c_p, _c_p]),
     "pa_prefill_workspace_size": (_c_sz, [_c_i32] * 5),
     "pa_prefill_varlen": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_i32, _c_p, _c_i32, _c_i32,
                                          _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_f32, _c_i32, _c_p, _c_sz, _c_p,
@@ -225,6 +228,16 @@ def pa_decode_split(out, q, k_cache, v_cache, block_table, context_lens, max_con
     """pa_decode with an explicit number of context splits (0 = automatic)."""
     pa_decode(out, q, k_cache, v_cache, block_table, context_lens, max_context_len, softmax_scale,
               workspace=workspace, dev_error=dev_error, stream=stream, num_splits=num_splits)
+
+
+def pa_decode_noalloc(out, q, k_cache, v_cache, block_table, context_lens, max_context_len, softmax_scale,
+                      dev_error=None, stream=None):
+    """pa_decode without a workspace: the split scratch is the library's fixed per-GPU array."""
+    nb, B, Hkv, D, batch, Hq, dev = _decode_args(out, q, k_cache, v_cache, block_table, context_lens)
+    _check(load_library().pa_decode_noalloc(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
+        _ptr(context_lens), batch, int(max_context_len), Hq, Hkv, D, nb, B, float(softmax_scale),
+        _opt_err(dev_error, dev), _stream(q, stream)))
 
 
 def pa_prefill_workspace_size(batch, max_seqlen_q, num_q_heads, num_kv_heads, head_dim) -> int:

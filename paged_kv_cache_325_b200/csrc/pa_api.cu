@@ -108,6 +108,10 @@ pa_status check_heads(int32_t num_q_heads, int32_t num_kv_heads) {
 
 }  // namespace
 
+namespace pa {
+void set_last_error(pa_status status, const char *detail) { fail(status, "%s", detail); }
+}  // namespace pa
+
 extern "C" {
 
 const char *pa_status_string(int status) {

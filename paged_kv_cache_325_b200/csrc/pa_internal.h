@@ -63,6 +63,10 @@ struct PrefillArgs {
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                            cudaStream_t stream);
 
+// ------------------------------------------------------------ error text --
+// Record the text pa_last_error_detail() returns on this thread.
+void set_last_error(pa_status status, const char *detail);
+
 // ------------------------------------------------------------- self-test --
 cudaError_t launch_selftest_wait(int32_t *dev_error, int64_t max_polls, cudaStream_t stream);
 

@@ -217,13 +217,15 @@ PA_API size_t pa_prefill_workspace_size(int32_t batch, int32_t max_seqlen_q, int
  *
  *   out[cu_q[s] + i, h] = sum_j softmax_j(softmax_scale * q[cu_q[s] + i, h] . K_j) V_j
  *
- *   out, q           [total_q, num_q_heads, head_dim] bf16, contiguous,
- *                    total_q = cu_seqlens_q[batch].
+ *   out, q           [total_q, num_q_heads, head_dim] bf16, contiguous;
+ *                    total_q (host) is their row count, >= cu_seqlens_q[batch]
+ *                    (checked mode reports a sequence that ends past it, and
+ *                    no row past it is ever read or written).
  *   cu_seqlens_q/k   [batch + 1] int32, device, starting at 0.
  *   max_seqlen_q/k   host-side upper bounds of n_new and n_k.
  *   block_table      [batch, block_table_stride] int32.
  */
-PA_API pa_status pa_prefill_varlen(void *out, const void *q, const void *k_cache, const void *v_cache,
+PA_API pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const void *k_cache, const void *v_cache,
                             const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t max_seqlen_q,
                             int32_t max_seqlen_k, const int32_t *block_table, int32_t block_table_stride,
                             int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,

@@ -62,7 +62,7 @@ _SIGS = {
     "pa_decode_noalloc": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_i32,
                                          _c_i32, _c_i32, _c_i32, _c_f32, _c_p, _c_p]),
     "pa_prefill_workspace_size": (_c_sz, [_c_i32] * 5),
-    "pa_prefill_varlen": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_i32, _c_p, _c_i32, _c_i32,
+    "pa_prefill_varlen": (ctypes.c_int, [_c_p, _c_p, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_i32, _c_p, _c_i32, _c_i32,
                                          _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_f32, _c_i32, _c_p, _c_sz, _c_p,
                                          _c_p]),
     "pa_selftest_bounded_wait": (ctypes.c_int, [_c_p, _c_i64, _c_p]),
@@ -262,7 +262,7 @@ def pa_prefill_varlen(out, q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_
         raise ValueError("cu_seqlens_q/k must be [batch+1] and block_table [batch, max_blocks]")
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load_library().pa_prefill_varlen(
-        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+        _ptr(out), _ptr(q), int(q.shape[0]), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
         int(max_seqlen_q), int(max_seqlen_k), _ptr(block_table), block_table.shape[1], batch, q.shape[1], Hkv, D,
         nb, B, float(softmax_scale), int(bool(causal)), _ptr(workspace), ws, _opt_err(dev_error, dev),
         _stream(q, stream)))

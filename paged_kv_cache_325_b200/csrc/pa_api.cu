@@ -269,7 +269,7 @@ size_t pa_prefill_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t nu
     return 0;
 }
 
-pa_status pa_prefill_varlen(void *out, const void *q, const void *k_cache, const void *v_cache,
+pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const void *k_cache, const void *v_cache,
                             const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t max_seqlen_q,
                             int32_t max_seqlen_k, const int32_t *block_table, int32_t block_table_stride,
                             int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
@@ -284,7 +284,8 @@ pa_status pa_prefill_varlen(void *out, const void *q, const void *k_cache, const
         return fail(PA_ERR_UNSUPPORTED, "prefill needs a GQA group that divides 128");
     if (!(softmax_scale > 0.f) || !isfinite(softmax_scale))
         return fail(PA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
-    if (batch == 0 || max_seqlen_q == 0) return ok();
+    if (total_q < 0) return fail(PA_ERR_INVALID_ARG, "total_q < 0");
+    if (batch == 0 || max_seqlen_q == 0 || total_q == 0) return ok();
     if (max_seqlen_q < 0 || max_seqlen_k < 1 || max_seqlen_k < max_seqlen_q)
         return fail(PA_ERR_INVALID_ARG, "need 0 <= max_seqlen_q <= max_seqlen_k and max_seqlen_k >= 1");
     if (block_table_stride < 1) return fail(PA_ERR_INVALID_ARG, "block_table_stride must be >= 1");
@@ -316,13 +317,17 @@ pa_status pa_prefill_varlen(void *out, const void *q, const void *k_cache, const
     a.max_seqlen_q = max_seqlen_q;
     a.max_seqlen_k = max_seqlen_k;
     a.causal = causal ? 1 : 0;
+    a.total_q = total_q;
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
 
     CUtensorMap tm_k, tm_v;
     const int64_t rows = (int64_t)num_blocks * block_size;
     if ((st = encode_rows(&tm_k, k_cache, rows, num_kv_heads, head_dim, 1, a.box_tokens)) != PA_OK) return st;
     if ((st = encode_rows(&tm_v, v_cache, rows, num_kv_heads, head_dim, 1, a.box_tokens)) != PA_OK) return st;
-    cudaError_t e = pa::launch_prefill(a, tm_k, tm_v, static_cast<cudaStream_t>(stream));
+    // q viewed as [total_q, Hq, D]: one box is the (128 / G) tokens x G q-heads of one Q tile
+    CUtensorMap tm_q;
+    if ((st = encode_rows(&tm_q, q, total_q, num_q_heads, head_dim, a.group, 128 / a.group)) != PA_OK) return st;
+    cudaError_t e = pa::launch_prefill(a, tm_q, tm_k, tm_v, static_cast<cudaStream_t>(stream));
     if (e == cudaErrorNotSupported) return fail(PA_ERR_UNSUPPORTED, "prefill kernel not available");
     if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
     return ok();

@@ -57,11 +57,11 @@ struct PrefillArgs {
     const int32_t *cu_q, *cu_k, *block_table;
     int32_t *dev_error;
     int32_t bt_stride, batch, num_q_heads, num_kv_heads, group, head_dim;
-    int32_t num_blocks, block_size, box_tokens, max_seqlen_q, max_seqlen_k, causal;
+    int32_t num_blocks, block_size, box_tokens, max_seqlen_q, max_seqlen_k, causal, total_q;
     float scale_log2;
 };
-cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                           cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                           const CUtensorMap &tm_v, cudaStream_t stream);
 
 // ------------------------------------------------------------ error text --
 // Record the text pa_last_error_detail() returns on this thread.

@@ -11,25 +11,29 @@
 // block table -- the flash_attn_varlen_func call of the nano-vllm walkthrough
 // (xingyun3d.csdn.net, sections seven and eight).
 //
-// How (one CTA per 128-row Q tile):
-//  * the 128 MMA rows are (128 / G) consecutive new tokens x the G q-heads
-//    of one KV head (GQA packing), so one K/V tile feeds all G heads;
-//  * warp 4 (TMA): K/V tiles of 128 keys, gathered block by block through
-//    block_table with 3-D tensor-map loads (128-byte swizzle), into a ring
-//    of shared-memory stages guarded by mbarriers;
-//  * warp 5 (MMA): one thread issues tcgen05.mma.cta_group::1.kind::f16:
-//    S = Q K^T (M=128, N=128, K=head_dim) into one of two TMEM S buffers,
-//    then O += P V (M=128, N=head_dim, K=128) into the TMEM O accumulator;
-//    tcgen05.commit signals the mbarriers;
-//  * warps 0-3 (softmax): thread t owns TMEM lane t, i.e. one Q row; it
-//    reads its S row with tcgen05.ld, selects masked keys out (-inf), keeps a
-//    running max in log2 units and rescales O (tcgen05.ld/st) only when the
-//    max grew by more than 8 (2^8), writes P as bf16 into a swizzled
-//    shared-memory tile (the A operand of the PV product), and at the end
-//    divides O by the row sum and stores bf16 rows to global memory;
-//  * V rows of the last key tile beyond the key range are zeroed in shared
-//    memory before the PV product, so stale or poisoned cache contents never
-//    meet a zero weight (0 * NaN is never formed).
+// How:
+//  * a Q tile is 128 MMA rows = (128 / G) consecutive new tokens x the G
+//    q-heads of one KV head (GQA packing), so one K/V tile feeds all G heads;
+//  * a work unit is two adjacent Q tiles (A, then B) of one (sequence, KV
+//    head); units are ordered by decreasing cost (last tiles of every sequence
+//    first) and dealt round-robin to persistent CTAs, one per SM;
+//  * warp 8 (TMA): per unit, both Q tiles (3-D tensor map over q), then the
+//    K and V tiles of 128 keys, gathered block by block through block_table,
+//    into a ring of shared-memory slots guarded by mbarriers;
+//  * warp 9 (MMA): one thread issues tcgen05.mma.cta_group::1.kind::f16 in the
+//    order S_A(0) S_B(0) | PV_A(j) S_A(j+1) PV_B(j) S_B(j+1) | ..., so the
+//    tensor cores work on one tile while the other tile's softmax runs.
+//    TMEM holds S_A, O_A, S_B, O_B (128 columns each); tcgen05.commit signals
+//    the mbarriers;
+//  * warps 0-3 / 4-7 (softmax of tile A / B): thread t owns TMEM lane t, i.e.
+//    one Q row; it reads its S row with tcgen05.ld, selects masked keys out
+//    (-inf), keeps a running max in log2 units and rescales O (tcgen05.ld/st)
+//    only when the max grew by more than 8 (2^8), writes P as bf16 into a
+//    swizzled shared-memory tile (the A operand of PV), and after the last key
+//    tile divides O by the row sum and stores bf16 rows;
+//  * V rows of a unit's last key tile beyond its key range are zeroed in
+//    shared memory before the PV products, so stale or poisoned cache contents
+//    never meet a zero weight (0 * NaN is never formed).
 #include <atomic>
 
 #include "pa_device.cuh"
@@ -39,114 +43,129 @@ namespace pa {
 
 namespace {
 
-constexpr int kM = 128;              // MMA rows per CTA
-constexpr int kN = 128;              // keys per K/V tile
-constexpr int kThreads = 192;        // 4 softmax warps + TMA warp + MMA warp
-constexpr int kTmaWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kRowBytes = 128;       // one 64-element bf16 swizzle row
-constexpr int kSlab = kM * kRowBytes;  // 128 rows x 128 B = 16 KB (a 64-column slice of a 128-row tile)
+constexpr int kM = 128;                // MMA rows per Q tile
+constexpr int kN = 128;                // keys per K/V tile
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;          // 2 softmax warpgroups + TMA warp + MMA warp
+constexpr int kRowBytes = 128;         // one 64-element bf16 swizzle row
+constexpr int kSlab = kM * kRowBytes;  // 128 rows x 128 B = 16 KB
 
 template <int D>
 struct PrefillCfg {
     static constexpr int kHalves = D / 64;
-    static constexpr int kStages = D == 128 ? 2 : 3;
-    static constexpr int kQBytes = kHalves * kSlab;
-    static constexpr int kKvBytes = kHalves * kSlab;          // one K (or V) tile of 128 keys
-    static constexpr int kStageBytes = 2 * kKvBytes;
-    static constexpr int kPBytes = 2 * kSlab;                 // P: 128 rows x 128 keys bf16
-    static constexpr int kQOff = 0;
-    static constexpr int kRingOff = kQOff + kQBytes;
-    static constexpr int kPOff = kRingOff + kStages * kStageBytes;
-    static constexpr int kBarOff = kPOff + kPBytes;
-    // barriers: kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full, pv_done, + tmem address slot
-    static constexpr int kNumBars = 2 * kStages + 6;
+    static constexpr int kSlots = D == 128 ? 3 : 6;             // K/V ring slots (one K or V tile each)
+    static constexpr int kTileBytes = kHalves * kSlab;          // a Q tile, or a K or V tile of 128 keys
+    static constexpr int kPBytes = 2 * kSlab;                   // P: 128 rows x 128 keys bf16
+    static constexpr int kQOff = 0;                             // Q_A, Q_B
+    static constexpr int kPOff = kQOff + 2 * kTileBytes;        // P_A, P_B
+    static constexpr int kRingOff = kPOff + 2 * kPBytes;
+    static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
+    // kv_full[S] kv_empty[S] q_full q_empty s_full[2] p_full[2] o_full[2] o_empty[2] done
+    static constexpr int kNumBars = 2 * kSlots + 11;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
-    static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+    static constexpr uint32_t kTmemCols = 512;                  // S_A 0, O_A 128, S_B 256, O_B 384
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
+
+__device__ __forceinline__ uint32_t col_s(int x) { return x ? 256u : 0u; }
+__device__ __forceinline__ uint32_t col_o(int x) { return x ? 384u : 128u; }
+
+struct Unit {
+    bool valid;
+    int s, kvh;
+    int q0;          // row of the sequence's first new token in q / out
+    int n_new, n_k, c;
+    int tok0[2];     // first new token of tile A / B (relative to the sequence)
+    int nq[2];       // tokens in tile A / B (0: tile absent)
+    int kend[2];     // keys [0, kend) visible to some row of the tile
+    int nt[2];       // key tiles of tile A / B
+    int nk;          // key tiles loaded for the unit
+};
+
+// Unit u of the cost-ordered list: rank r = u / (batch * Hkv) counts pairs of
+// Q tiles from the end of each sequence (r = 0: the last, longest pair).
+__device__ __forceinline__ Unit unit_of(const PrefillArgs &a, int u, int TQ) {
+    Unit U;
+    U.valid = false;
+    const int per_rank = a.batch * a.num_kv_heads;
+    const int r = u / per_rank, sk = u % per_rank;
+    U.s = sk / a.num_kv_heads;
+    U.kvh = sk % a.num_kv_heads;
+    const int q0 = __ldg(a.cu_q + U.s), q1 = __ldg(a.cu_q + U.s + 1);
+    const int k0 = __ldg(a.cu_k + U.s), k1 = __ldg(a.cu_k + U.s + 1);
+    U.n_new = q1 - q0;
+    U.n_k = k1 - k0;
+    U.c = U.n_k - U.n_new;
+    if (U.n_new < 0 || U.c < 0 || q0 < 0 || k0 < 0 || q1 > a.total_q || U.n_new > a.max_seqlen_q ||
+        U.n_k > a.max_seqlen_k || (int64_t)U.n_k > (int64_t)a.bt_stride * a.block_size) {
+        if (r == 0 && U.kvh == 0 && threadIdx.x == 0) report(a.dev_error, PA_DEVERR_SEQLENS);
+        return U;
+    }
+    const int npairs = (U.n_new + 2 * TQ - 1) / (2 * TQ);
+    if (r >= npairs) return U;
+    const int p = npairs - 1 - r;
+    U.q0 = q0;
+    for (int x = 0; x < 2; ++x) {
+        U.tok0[x] = (2 * p + x) * TQ;
+        U.nq[x] = max(0, min(TQ, U.n_new - U.tok0[x]));
+        U.kend[x] = U.nq[x] == 0 ? 0 : (a.causal ? U.c + U.tok0[x] + U.nq[x] : U.n_k);
+        U.nt[x] = (U.kend[x] + kN - 1) / kN;
+    }
+    U.nk = max(U.nt[0], U.nt[1]);
+    U.valid = true;
+    return U;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const PrefillArgs a) {
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
     using C = PrefillCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *kv_full = bars;
-    uint64_t *kv_empty = bars + C::kStages;
-    uint64_t *s_full = bars + 2 * C::kStages;
-    uint64_t *s_free = s_full + 2;
-    uint64_t *p_full = s_free + 2;
-    uint64_t *pv_done = p_full + 1;
+    uint64_t *kv_empty = bars + C::kSlots;
+    uint64_t *q_full = bars + 2 * C::kSlots;
+    uint64_t *q_empty = q_full + 1;
+    uint64_t *s_full = q_empty + 1;    // [2]
+    uint64_t *p_full = s_full + 2;     // [2]
+    uint64_t *o_full = p_full + 2;     // [2]
+    uint64_t *o_empty = o_full + 2;    // [2]
+    uint64_t *done = o_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.group;
-    const int TQ = kM / G;                        // tokens per Q tile
-    const int kvh = blockIdx.x % a.num_kv_heads;
-    const int s = blockIdx.x / a.num_kv_heads;
-
-    // ---- sequence geometry (validated; a bad sequence is skipped) ----
-    const int q0 = __ldg(a.cu_q + s), q1 = __ldg(a.cu_q + s + 1);
-    const int k0 = __ldg(a.cu_k + s), k1 = __ldg(a.cu_k + s + 1);
-    const int n_new = q1 - q0, n_k = k1 - k0, c = n_k - n_new;
-    if (n_new < 0 || c < 0 || q0 < 0 || k0 < 0 || n_new > a.max_seqlen_q || n_k > a.max_seqlen_k ||
-        (int64_t)n_k > (int64_t)a.bt_stride * a.block_size) {
-        if (blockIdx.y == 0 && kvh == 0 && threadIdx.x == 0) report(a.dev_error, PA_DEVERR_SEQLENS);
-        return;
-    }
-    const int nqt = (n_new + TQ - 1) / TQ;
-    if ((int)blockIdx.y >= nqt) return;
-    const int qt = nqt - 1 - (int)blockIdx.y;    // blockIdx.y = 0 takes the last (longest) tile
-    const int tok0 = qt * TQ;                    // first new token of this tile
-    const int nq = min(TQ, n_new - tok0);
-    const int kend = a.causal ? c + tok0 + nq : n_k;   // keys [0, kend) are visible to some row
-    const int nkt = (kend + kN - 1) / kN;
+    const int TQ = kM / G;
+    const int per_rank = a.batch * a.num_kv_heads;
+    const int num_units = ((a.max_seqlen_q + 2 * TQ - 1) / (2 * TQ)) * per_rank;
 
     const uint32_t sbase = smem_u32(smem);
     const uint32_t q_s = sbase + C::kQOff;
-    const uint32_t ring = sbase + C::kRingOff;
     const uint32_t p_s = sbase + C::kPOff;
+    const uint32_t ring = sbase + C::kRingOff;
 
-    // ---- barriers and TMEM ----
     if (threadIdx.x == 0) {
-        for (int st = 0; st < C::kStages; ++st) {
-            mbar_init(smem_u32(kv_full + st), 1);
-            mbar_init(smem_u32(kv_empty + st), 1);
+        for (int i = 0; i < C::kSlots; ++i) {
+            mbar_init(smem_u32(kv_full + i), 1);
+            mbar_init(smem_u32(kv_empty + i), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(smem_u32(s_full + b), 1);
-            mbar_init(smem_u32(s_free + b), 4);
+        mbar_init(smem_u32(q_full), 1);
+        mbar_init(smem_u32(q_empty), 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(smem_u32(s_full + x), 1);
+            mbar_init(smem_u32(p_full + x), 4);
+            mbar_init(smem_u32(o_full + x), 1);
+            mbar_init(smem_u32(o_empty + x), 4);
         }
-        mbar_init(smem_u32(p_full), 4);
-        mbar_init(smem_u32(pv_done), 1);
+        mbar_init(smem_u32(done), 1);
         fence_barrier_init();
     }
     if (warp == kMmaWarp) {
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
-    }
-
-    // ---- Q tile -> shared memory (K-major, 128-byte swizzle), zero rows past n_new ----
-    {
-        const uint16_t *qg = static_cast<const uint16_t *>(a.q);
-        constexpr int kChunksPerRow = D / 8;
-        for (int e = threadIdx.x; e < kM * kChunksPerRow; e += kThreads) {
-            const int r = e / kChunksPerRow, ch = e % kChunksPerRow;
-            const int t = tok0 + r / G;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t < n_new) {
-                const int64_t row = ((int64_t)(q0 + t) * a.num_q_heads + (int64_t)kvh * G + r % G) * D;
-                v = __ldg(reinterpret_cast<const uint4 *>(qg + row) + ch);
-            }
-            const uint32_t dst = q_s + (ch >> 3) * kSlab + swz128(r, ch & 7);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
-                         "r"(v.w)
-                         : "memory");
-        }
-        fence_proxy_async_smem();   // make the generic-proxy writes visible to the tensor cores
     }
     tc_fence_before();
     __syncthreads();
@@ -156,35 +175,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kTmaWarp) {
         // ============================================================ TMA ==
         if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            const int32_t *bt = a.block_table + (int64_t)s * a.bt_stride;
             const int B = a.block_size, box = a.box_tokens;
-            for (int j = 0; j < nkt; ++j) {
-                const int st = j % C::kStages;
-                if (j >= C::kStages &&
-                    !mbar_wait(smem_u32(kv_empty + st), ((j / C::kStages) & 1) ^ 1, a.dev_error))
-                    break;
-                const int key0 = j * kN;
-                const int nbox = (min(kN, kend - key0) + box - 1) / box;
-                const uint32_t fb = smem_u32(kv_full + st);
-                mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * kRowBytes * C::kHalves * 2));
-                const uint32_t kd = ring + st * C::kStageBytes, vd = kd + C::kKvBytes;
-                for (int b = 0; b < nbox; ++b) {
-                    const int tok = key0 + b * box;
-                    const int blk = __ldg(bt + tok / B);
-                    int row;
-                    if ((unsigned)blk < (unsigned)a.num_blocks) {
-                        row = blk * B + (tok % B);
-                    } else {
-                        report(a.dev_error, PA_DEVERR_BLOCK_ID);
-                        row = -box;          // fully out of range: TMA fills zeros
-                    }
+            uint32_t nq = 0, L = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+                const Unit U = unit_of(a, u, TQ);
+                if (!U.valid) continue;
+                if (nq > 0 && !mbar_wait(smem_u32(q_empty), (nq - 1) & 1, a.dev_error)) break;
+                mbar_arrive_expect_tx(smem_u32(q_full), (uint32_t)(2 * C::kTileBytes));
+                for (int x = 0; x < 2; ++x)
 #pragma unroll
-                    for (int h = 0; h < C::kHalves; ++h) {
-                        const uint32_t off = h * kSlab + b * box * kRowBytes;
-                        tma_load_3d(kd + off, &tm_k, h * 64, kvh, row, fb);
-                        tma_load_3d(vd + off, &tm_v, h * 64, kvh, row, fb);
+                    for (int h = 0; h < C::kHalves; ++h)
+                        tma_load_3d(q_s + x * C::kTileBytes + h * kSlab, &tm_q, h * 64, U.kvh * G,
+                                    U.q0 + U.tok0[x], smem_u32(q_full));
+                ++nq;
+                const int32_t *bt = a.block_table + (int64_t)U.s * a.bt_stride;
+                const int kend = max(U.kend[0], U.kend[1]);
+                for (int j = 0; j < U.nk && ok; ++j) {
+                    const int key0 = j * kN;
+                    const int nbox = (min(kN, kend - key0) + box - 1) / box;
+                    for (int kv = 0; kv < 2; ++kv, ++L) {
+                        const int slot = L % C::kSlots;
+                        if (L >= (uint32_t)C::kSlots &&
+                            !mbar_wait(smem_u32(kv_empty + slot), (L / C::kSlots - 1) & 1, a.dev_error)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t fb = smem_u32(kv_full + slot);
+                        mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * kRowBytes * C::kHalves));
+                        const uint32_t dst = ring + slot * C::kTileBytes;
+                        for (int b = 0; b < nbox; ++b) {
+                            const int tok = key0 + b * box;
+                            const int blk = __ldg(bt + tok / B);
+                            int row;
+                            if ((unsigned)blk < (unsigned)a.num_blocks) {
+                                row = blk * B + (tok % B);
+                            } else {
+                                report(a.dev_error, PA_DEVERR_BLOCK_ID);
+                                row = -box;     // fully out of range: TMA fills zeros
+                            }
+#pragma unroll
+                            for (int h = 0; h < C::kHalves; ++h)
+                                tma_load_3d(dst + h * kSlab + b * box * kRowBytes, kv ? &tm_v : &tm_k, h * 64, U.kvh,
+                                            row, fb);
+                        }
                     }
                 }
             }
@@ -193,160 +230,206 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ============================================================ MMA ==
         constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kN, 0, 0);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, D, 0, 1);
+        uint32_t nq = 0, L = 0, np[2] = {0, 0}, no[2] = {0, 0};
         bool ok = true;
-        auto issue_pv = [&](int jj) -> bool {
-            const int st = jj % C::kStages;
-            if (!mbar_wait(smem_u32(p_full), jj & 1, a.dev_error)) return false;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t vs = ring + st * C::kStageBytes + C::kKvBytes;
-#pragma unroll
-                for (int kk = 0; kk < kN / 16; ++kk) {
-                    // A = P rows, K-major: key half kk/4, 32-byte step inside the swizzle row
-                    const uint64_t ad = smem_desc_sw128(p_s + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
-                    // B = V, MN-major: 16 keys = 2 groups of 8 rows; the D halves are kSlab apart
-                    const uint64_t bd = smem_desc_sw128(vs + kk * 16 * kRowBytes, kSlab, 1024);
-                    tc_mma_ss(tmem + C::kColO, ad, bd, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-                }
-                tc_commit(smem_u32(kv_empty + st));
-                tc_commit(smem_u32(pv_done));
-            }
-            __syncwarp();
-            return true;
+        auto wait_slot = [&](uint32_t idx) -> bool {
+            return mbar_wait(smem_u32(kv_full + idx % C::kSlots), (idx / C::kSlots) & 1, a.dev_error);
         };
-        for (int j = 0; j < nkt && ok; ++j) {
-            const int st = j % C::kStages, b = j & 1;
-            if (!mbar_wait(smem_u32(kv_full + st), (j / C::kStages) & 1, a.dev_error)) { ok = false; break; }
-            if (j >= 2 && !mbar_wait(smem_u32(s_free + b), ((j >> 1) - 1) & 1, a.dev_error)) { ok = false; break; }
-            // last tile: zero the V rows past the key range (stale or poisoned slots)
-            const int valid = kend - j * kN;
-            if (valid < kN) {
-                const uint32_t vs = ring + st * C::kStageBytes + C::kKvBytes;
-                for (int e = lane; e < (kN - valid) * C::kHalves * 8; e += 32) {
-                    const int r = valid + e / (C::kHalves * 8);
-                    const int h = (e / 8) % C::kHalves, ch = e % 8;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(vs + h * kSlab + r * kRowBytes +
-                                                                                   ch * 16),
-                                 "r"(0u)
-                                 : "memory");
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-            }
-            tc_fence_after();
+        auto issue_s = [&](int x, uint32_t kidx) {
             if (lane == 0) {
-                const uint32_t ks = ring + st * C::kStageBytes;
+                const uint32_t ks = ring + (kidx % C::kSlots) * C::kTileBytes;
+                const uint32_t qs = q_s + x * C::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(q_s + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
+                    const uint64_t ad = smem_desc_sw128(qs + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
                     const uint64_t bd = smem_desc_sw128(ks + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
-                    tc_mma_ss(tmem + (b ? C::kColS1 : C::kColS0), ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    tc_mma_ss(tmem + col_s(x), ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                tc_commit(smem_u32(s_full + b));
+                tc_commit(smem_u32(s_full + x));
             }
             __syncwarp();
-            if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        };
+        auto issue_pv = [&](int x, uint32_t vidx, bool accumulate) {
+            if (lane == 0) {
+                const uint32_t vs = ring + (vidx % C::kSlots) * C::kTileBytes;
+                const uint32_t ps = p_s + x * C::kPBytes;
+#pragma unroll
+                for (int kk = 0; kk < kN / 16; ++kk) {
+                    const uint64_t ad = smem_desc_sw128(ps + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(vs + kk * 16 * kRowBytes, kSlab, 1024);
+                    tc_mma_ss(tmem + col_o(x), ad, bd, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+                }
+            }
+            __syncwarp();
+        };
+        auto commit = [&](uint64_t *bar) {
+            if (lane == 0) tc_commit(smem_u32(bar));
+            __syncwarp();
+        };
+        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            const Unit U = unit_of(a, u, TQ);
+            if (!U.valid) continue;
+            if (!mbar_wait(smem_u32(q_full), nq & 1, a.dev_error)) break;
+            ++nq;
+            const bool hasB = U.nt[1] > 0;
+            // K_0: S_A(0), S_B(0)
+            if (!wait_slot(L)) break;
+            tc_fence_after();
+            issue_s(0, L);
+            if (hasB) issue_s(1, L);
+            commit(kv_empty + L % C::kSlots);
+            if (U.nk == 1) commit(q_empty);
+            for (int j = 0; j < U.nk && ok; ++j) {
+                const uint32_t vidx = L + 2 * j + 1, knext = L + 2 * j + 2;
+                if (!wait_slot(vidx)) { ok = false; break; }
+                if (j == U.nk - 1) {
+                    // zero V rows past the unit's key range (stale or poisoned slots)
+                    const int valid = max(U.kend[0], U.kend[1]) - j * kN;
+                    if (valid < kN) {
+                        const uint32_t vs = ring + (vidx % C::kSlots) * C::kTileBytes;
+                        for (int e = lane; e < (kN - valid) * C::kHalves * 8; e += 32) {
+                            const int r = valid + e / (C::kHalves * 8);
+                            const int h = (e / 8) % C::kHalves, ch = e % 8;
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(
+                                             vs + h * kSlab + r * kRowBytes + ch * 16),
+                                         "r"(0u)
+                                         : "memory");
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                    }
+                }
+                bool knext_ready = false;
+                for (int x = 0; x < 2; ++x) {
+                    if (j >= U.nt[x]) continue;
+                    if (!mbar_wait(smem_u32(p_full + x), np[x] & 1, a.dev_error)) { ok = false; break; }
+                    ++np[x];
+                    if (j == 0 && no[x] > 0 && !mbar_wait(smem_u32(o_empty + x), (no[x] - 1) & 1, a.dev_error)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_pv(x, vidx, j > 0);
+                    if (j == U.nt[x] - 1) {
+                        commit(o_full + x);
+                        ++no[x];
+                    }
+                    if (j + 1 < U.nt[x]) {
+                        if (!knext_ready) {
+                            if (!wait_slot(knext)) { ok = false; break; }
+                            tc_fence_after();
+                            knext_ready = true;
+                        }
+                        issue_s(x, knext);
+                    }
+                }
+                if (!ok) break;
+                commit(kv_empty + vidx % C::kSlots);
+                if (knext_ready) commit(kv_empty + knext % C::kSlots);
+                if (j == U.nk - 2) commit(q_empty);   // every S product of the unit is issued
+            }
+            L += 2 * U.nk;
         }
-        if (ok && nkt > 0) issue_pv(nkt - 1);
+        // every MMA issued by this thread has completed before TMEM is freed
+        commit(done);
+        mbar_wait(smem_u32(done), 0, a.dev_error);
     } else {
         // ======================================================== softmax ==
-        const int r = threadIdx.x;                      // TMEM lane == Q-tile row
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-        const int t = tok0 + r / G;                     // this row's new-token index
-        int lim = a.causal ? c + t : n_k - 1;           // last visible key
-        if (lim > n_k - 1) lim = n_k - 1;               // rows past n_new never see past the keys
-        float m_ref = -INFINITY, l = 0.f;
-        bool ok = true;
-        for (int j = 0; j < nkt; ++j) {
-            const int b = j & 1;
-            if (!mbar_wait(smem_u32(s_full + b), (j >> 1) & 1, a.dev_error)) { ok = false; break; }
-            tc_fence_after();
-            float sv[kN];
-            {
-                uint32_t raw[32];
-#pragma unroll
-                for (int q = 0; q < kN / 32; ++q) {
-                    tmem_ld32(lane_base + (b ? C::kColS1 : C::kColS0) + q * 32, raw);
-                    tc_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) sv[q * 32 + e] = __uint_as_float(raw[e]);
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(s_free + b));
-
-            const int key0 = j * kN;
-            float mt = -INFINITY;
-            if (key0 + kN - 1 <= lim) {
-#pragma unroll
-                for (int e = 0; e < kN; ++e) {
-                    sv[e] *= a.scale_log2;
-                    mt = fmaxf(mt, sv[e]);
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < kN; ++e) {
-                    sv[e] = (key0 + e <= lim) ? sv[e] * a.scale_log2 : -INFINITY;
-                    mt = fmaxf(mt, sv[e]);
-                }
-            }
-            bool rescale = false;
-            float corr = 1.f;
-            if (mt > m_ref + 8.f) {                     // also true while m_ref is -inf
-                corr = fast_exp2(m_ref - mt);
-                m_ref = mt;
-                rescale = true;
-            }
-            l *= corr;
-            uint32_t pk[kN / 2];
-#pragma unroll
-            for (int e = 0; e < kN; e += 2) {
-                const float p0 = fast_exp2(sv[e] - m_ref);
-                const float p1 = fast_exp2(sv[e + 1] - m_ref);
-                pk[e / 2] = pack_bf16(p0, p1);
-                const __nv_bfloat162 pb = *reinterpret_cast<const __nv_bfloat162 *>(&pk[e / 2]);
-                l += __low2float(pb) + __high2float(pb);
-            }
-            // the previous PV product must be done before P and O are touched
-            if (j >= 1 && !mbar_wait(smem_u32(pv_done), (j - 1) & 1, a.dev_error)) { ok = false; break; }
-            if (rescale && j >= 1) {
+        const int x = warp >> 2;                       // 0: tile A, 1: tile B
+        const int r = threadIdx.x & 127;               // TMEM lane == Q-tile row
+        const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const float sl = a.scale_log2;
+        uint32_t ns = 0, no = 0;
+        for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+            const Unit U = unit_of(a, u, TQ);
+            if (!U.valid || U.nt[x] == 0) continue;
+            const int t = U.tok0[x] + r / G;              // this row's new-token index
+            int lim = a.causal ? U.c + t : U.n_k - 1;      // last visible key
+            if (lim > U.n_k - 1) lim = U.n_k - 1;          // rows past n_new never see past the keys
+            float m_ref = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < U.nt[x]; ++j) {
+                if (!mbar_wait(smem_u32(s_full + x), ns & 1, a.dev_error)) { ok = false; break; }
+                ++ns;
                 tc_fence_after();
+                uint32_t sr[4][32];
 #pragma unroll
-                for (int q = 0; q < D / 32; ++q) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_base + C::kColO + q * 32, o);
-                    tc_wait_ld();
+                for (int q = 0; q < 4; ++q) tmem_ld32(lane_base + col_s(x) + q * 32, sr[q]);
+                tc_wait_ld();
+                const int thr = lim - j * kN;              // keys e <= thr are visible
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if (thr >= kN - 1) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-                    tmem_st32(lane_base + C::kColO + q * 32, o);
+                    for (int e = 0; e < kN; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(sr[e >> 5][e & 31]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < kN; ++e) {
+                        const float v = e <= thr ? __uint_as_float(sr[e >> 5][e & 31]) : -INFINITY;
+                        sr[e >> 5][e & 31] = __float_as_uint(v);
+                        mx[e & 3] = fmaxf(mx[e & 3], v);
+                    }
                 }
-                tc_wait_st();
-            }
+                const float m_new = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl;
+                float corr = 1.f;
+                bool rescale = false;
+                if (m_new > m_ref + 8.f) {                  // also true while m_ref is -inf
+                    corr = fast_exp2(m_ref - m_new);
+                    m_ref = m_new;
+                    rescale = true;
+                }
+                const float neg = -m_ref;
+                // P = exp2(s * scale_log2 - m_ref) as bf16, stored 8 keys (16 bytes) at a time
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint32_t pb = p_s + x * C::kPBytes;
 #pragma unroll
-            for (int kc = 0; kc < kN / 8; ++kc) {
-                const uint32_t dst = p_s + (kc >> 3) * kSlab + swz128(r, kc & 7);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[kc * 4]),
-                             "r"(pk[kc * 4 + 1]), "r"(pk[kc * 4 + 2]), "r"(pk[kc * 4 + 3])
-                             : "memory");
+                for (int kc = 0; kc < kN / 8; ++kc) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int e = kc * 8 + 2 * i;
+                        const float p0 = fast_exp2(fmaf(__uint_as_float(sr[e >> 5][e & 31]), sl, neg));
+                        const float p1 = fast_exp2(fmaf(__uint_as_float(sr[e >> 5][(e + 1) & 31]), sl, neg));
+                        w[i] = pack_bf16(p0, p1);
+                        ls[i] += p0 + p1;
+                    }
+                    const uint32_t dst = pb + (kc >> 3) * kSlab + swz128(r, kc & 7);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w[0]), "r"(w[1]),
+                                 "r"(w[2]), "r"(w[3])
+                                 : "memory");
+                }
+                l = l * corr + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+                if (rescale && j > 0) {
+                    // O_X is stable: PV_X(j-1) completed before S_X(j), which was issued after it
+#pragma unroll
+                    for (int q = 0; q < D / 32; ++q) {
+                        uint32_t o[32];
+                        tmem_ld32(lane_base + col_o(x) + q * 32, o);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+                        tmem_st32(lane_base + col_o(x) + q * 32, o);
+                    }
+                    tc_wait_st();
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(p_full + x));
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(p_full));
-        }
-        // ---- epilogue: O / l -> bf16 rows ----
-        if (ok && nkt > 0 && mbar_wait(smem_u32(pv_done), (nkt - 1) & 1, a.dev_error)) {
+            if (!ok) break;
+            // ---- epilogue: O / l -> bf16 rows ----
+            if (!mbar_wait(smem_u32(o_full + x), no & 1, a.dev_error)) break;
+            ++no;
             tc_fence_after();
             const float inv = 1.f / l;
-            const bool store = t < n_new;
+            const bool store = t < U.n_new;
             uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) +
-                                                   ((int64_t)(q0 + (store ? t : 0)) * a.num_q_heads +
-                                                    (int64_t)kvh * G + r % G) * D);
+                                                   ((int64_t)(U.q0 + (store ? t : 0)) * a.num_q_heads +
+                                                    (int64_t)U.kvh * G + r % G) * D);
 #pragma unroll
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t o[32];
-                tmem_ld32(lane_base + C::kColO + q * 32, o);
+                tmem_ld32(lane_base + col_o(x) + q * 32, o);
                 tc_wait_ld();
                 if (store) {
 #pragma unroll
@@ -360,6 +443,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(o_empty + x));
         }
     }
 
@@ -371,9 +457,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
 template <int D>
-cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                             cudaStream_t stream) {
+cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                             const CUtensorMap &tm_v, cudaStream_t stream) {
     using C = PrefillCfg<D>;
     static std::atomic<uint64_t> configured{0};
     int dev = 0;
@@ -386,17 +479,19 @@ cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &tm_k, cons
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
     const int TQ = kM / a.group;
-    const dim3 grid((unsigned)(a.batch * a.num_kv_heads), (unsigned)((a.max_seqlen_q + TQ - 1) / TQ));
-    prefill_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tm_k, tm_v, a);
+    const int64_t units = (int64_t)((a.max_seqlen_q + 2 * TQ - 1) / (2 * TQ)) * a.batch * a.num_kv_heads;
+    const int grid = (int)(units < num_sms() ? units : num_sms());
+    if (grid <= 0) return cudaSuccess;
+    prefill_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tm_q, tm_k, tm_v, a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
-                           cudaStream_t stream) {
-    if (a.head_dim == 128) return launch_prefill_d<128>(a, tm_k, tm_v, stream);
-    return launch_prefill_d<64>(a, tm_k, tm_v, stream);
+cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                           const CUtensorMap &tm_v, cudaStream_t stream) {
+    if (a.head_dim == 128) return launch_prefill_d<128>(a, tm_q, tm_k, tm_v, stream);
+    return launch_prefill_d<64>(a, tm_q, tm_k, tm_v, stream);
 }
 
 }  // namespace pa

@@ -97,10 +97,10 @@ def test_decode_workspace_size_query():
 
 
 def _prefill(lib, **kw):
-    a = dict(out=A, q=A, kc=A, vc=A, cq=A, ck=A, mq=100, mk=200, bt=A, bts=4, batch=2, Hq=32, Hkv=8, D=128,
+    a = dict(out=A, q=A, tq=150, kc=A, vc=A, cq=A, ck=A, mq=100, mk=200, bt=A, bts=4, batch=2, Hq=32, Hkv=8, D=128,
              nb=16, B=256, scale=0.088, causal=1, err=None)
     a.update(kw)
-    return lib.pa_prefill_varlen(a["out"], a["q"], a["kc"], a["vc"], a["cq"], a["ck"], a["mq"], a["mk"], a["bt"],
+    return lib.pa_prefill_varlen(a["out"], a["q"], a["tq"], a["kc"], a["vc"], a["cq"], a["ck"], a["mq"], a["mk"], a["bt"],
                                  a["bts"], a["batch"], a["Hq"], a["Hkv"], a["D"], a["nb"], a["B"], a["scale"],
                                  a["causal"], None, 0, a["err"], None)
 
@@ -113,6 +113,8 @@ def test_prefill_validation(lib):
     assert _prefill(lib, ck=P(0x10001)) == pa.PA_ERR_INVALID_ARG
     assert _prefill(lib, batch=0) == pa.PA_OK
     assert _prefill(lib, mq=0) == pa.PA_OK
+    assert _prefill(lib, tq=0) == pa.PA_OK
+    assert _prefill(lib, tq=-1) == pa.PA_ERR_INVALID_ARG
 
 
 def test_selftest_validation(lib):

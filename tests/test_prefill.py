@@ -113,3 +113,25 @@ def test_prefill_checked_mode(cuda_lib):
     g.prefill(dev_error=err)
     torch.cuda.synchronize()
     assert int(err.item()) & pa.PA_DEVERR_SEQLENS
+
+
+def test_prefill_many_sequences_exercise_persistent_units(cuda_lib):
+    """Far more work units than SMs: every CTA walks many units, carrying its
+    barrier phases and TMEM buffers from one unit to the next."""
+    rng = np.random.default_rng(31)
+    L = rng.integers(1, 400, size=180)
+    c = np.array([(int(x) - 1) // 64 * 64 if i % 3 == 0 else 0 for i, x in enumerate(L)])
+    case = W.make_prefill_case(L, c, 16, 4, 128, 64, seed=961)
+    _, out = _run(case)
+    assert_close(out, oracle_prefill(case), what="180 sequences")
+
+
+def test_prefill_head_dim_64_long_prompt(cuda_lib):
+    case = W.make_prefill_case([1500, 700], [1024, 0], 32, 8, 64, 256, seed=962)
+    _, out = _run(case)
+    rng = np.random.default_rng(2)
+    toks = rng.integers(0, case.total_q, size=1500)
+    heads = rng.integers(0, 32, size=1500)
+    ref = oracle_prefill(case, tok_idx=toks, head_idx=heads)
+    assert_close(out[torch.tensor(toks), torch.tensor(heads)], ref, what="D=64 long prompt")
+    assert torch.isfinite(out.float()).all()

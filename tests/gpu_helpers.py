@@ -7,7 +7,10 @@ import oracle
 import paged_kv_cache_325_b200 as pa
 
 # Tolerance of the attention outputs against the fp64 oracle (bf16 in, fp32
-# accumulate, bf16 out): worst element and mean over all elements.
+# accumulate, bf16 out): max-abs 1e-2 and mean-abs 1e-3.  The output itself is
+# bf16, whose rounding alone is up to half an ulp (2^-9 relative; 0.0156 for
+# |x| in [4, 8)), so the max-abs bar applies to the error beyond that rounding:
+# |gpu - ref| <= 1e-2 + ulp_bf16(ref) / 2 elementwise.
 MAX_ABS = 1e-2
 MEAN_ABS = 1e-3
 
@@ -16,11 +19,19 @@ def i32(a, dev):
     return torch.as_tensor(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
 
 
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 numbers at |x| (8 significant bits)."""
+    _, e = np.frexp(np.abs(x))                # |x| = m * 2^e, m in [0.5, 1)
+    return np.where(x == 0, 0.0, np.ldexp(1.0, e - 9))
+
+
 def assert_close(gpu_bf16: torch.Tensor, ref: np.ndarray, max_abs=MAX_ABS, mean_abs=MEAN_ABS, what=""):
     g = gpu_bf16.detach().to("cpu", torch.float64).numpy().reshape(ref.shape)
     assert np.isfinite(g).all(), f"{what}: non-finite GPU output"
     err = np.abs(g - ref)
-    assert err.max() <= max_abs, f"{what}: max abs err {err.max():.3e} > {max_abs}"
+    excess = err - bf16_half_ulp(ref)
+    assert excess.max() <= max_abs, (f"{what}: error beyond bf16 output rounding {excess.max():.3e} > {max_abs} "
+                                     f"(raw max abs {err.max():.3e})")
     assert err.mean() <= mean_abs, f"{what}: mean abs err {err.mean():.3e} > {mean_abs}"
     return float(err.max()), float(err.mean())
 

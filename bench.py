@@ -359,12 +359,14 @@ def bench_secondary(args, device, pk, names):
     cq = torch.as_tensor(case.cu_seqlens_q).to(dev)
     ck = torch.as_tensor(case.cu_seqlens_k).to(dev)
     o = torch.empty_like(q)
+    pws = pa.alloc_prefill_workspace(q, case.num_kv_heads, case.batch, case.max_seqlen_q)
 
     def st():
         pa.pa_store_kv(kn, vn, slot, kc, vc)
 
     def pf():
-        pa.pa_prefill_varlen(o, q, kc, vc, cq, ck, case.max_seqlen_q, case.max_seqlen_k, bt, case.softmax_scale)
+        pa.pa_prefill_varlen(o, q, kc, vc, cq, ck, case.max_seqlen_q, case.max_seqlen_k, bt, case.softmax_scale,
+                             workspace=pws)
 
     st_replay, _g1 = capture(st)
     pf_replay, _g2 = capture(pf)

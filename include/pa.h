@@ -199,7 +199,12 @@ PA_API pa_status pa_decode_noalloc(void *out, const void *q, const void *k_cache
                                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
                                    int32_t block_size, float softmax_scale, int32_t *dev_error, void *stream);
 
-/* Bytes of device workspace pa_prefill_varlen needs (currently always 0). */
+/*
+ * Bytes of device workspace pa_prefill_varlen needs: a table of the work units
+ * (pairs of 128-row Q tiles), ordered from the most to the least expensive,
+ * and the counter the persistent kernel hands them out with.  It grows with
+ * batch and max_seqlen_q (a few KB for a dozen prompts of 2k tokens).
+ */
 PA_API size_t pa_prefill_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t num_q_heads,
                                  int32_t num_kv_heads, int32_t head_dim);
 
@@ -224,6 +229,14 @@ PA_API size_t pa_prefill_workspace_size(int32_t batch, int32_t max_seqlen_q, int
  *   cu_seqlens_q/k   [batch + 1] int32, device, starting at 0.
  *   max_seqlen_q/k   host-side upper bounds of n_new and n_k.
  *   block_table      [batch, block_table_stride] int32.
+ *   workspace        device scratch of at least pa_prefill_workspace_size()
+ *                    bytes, 256-byte aligned; no initialisation needed (a
+ *                    planning kernel on the same stream rewrites it every call),
+ *                    garbage afterwards.  batch <= 6144.
+ *
+ * Two kernels run: a one-CTA planning kernel that validates every sequence and
+ * orders the work units, then the persistent prefill kernel (launched with
+ * programmatic dependent launch so its prologue overlaps the planning).
  */
 PA_API pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const void *k_cache, const void *v_cache,
                             const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t max_seqlen_q,

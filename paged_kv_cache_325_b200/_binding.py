@@ -35,7 +35,7 @@ PA_DEVERR_TIMEOUT = 0x10
 __all__ = ["PagedAttnError", "load_library", "declared_symbols", "pa_store_kv", "pa_decode", "pa_decode_split",
            "pa_decode_workspace_size", "pa_decode_split_workspace_size", "pa_decode_noalloc", "pa_prefill_varlen",
            "pa_prefill_workspace_size", "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
-           "alloc_decode_workspace"]
+           "alloc_decode_workspace", "alloc_prefill_workspace"]
 
 
 class PagedAttnError(RuntimeError):
@@ -244,9 +244,18 @@ def pa_prefill_workspace_size(batch, max_seqlen_q, num_q_heads, num_kv_heads, he
     return int(load_library().pa_prefill_workspace_size(batch, max_seqlen_q, num_q_heads, num_kv_heads, head_dim))
 
 
+def alloc_prefill_workspace(q, num_kv_heads, batch, max_seqlen_q):
+    """A torch-owned workspace of the size pa_prefill_varlen needs (its work-unit table)."""
+    import torch
+    n = pa_prefill_workspace_size(batch, max_seqlen_q, q.shape[1], num_kv_heads, q.shape[2])
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+
+
 def pa_prefill_varlen(out, q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
                       block_table, softmax_scale, causal=True, workspace=None, dev_error=None, stream=None):
-    """Varlen (causal) prefill over the paged cache into `out` ([total_q, Hq, D] bf16)."""
+    """Varlen (causal) prefill over the paged cache into `out` ([total_q, Hq, D] bf16).
+
+    `workspace`: device scratch of pa_prefill_workspace_size() bytes (alloc_prefill_workspace)."""
     import torch
     nb, B, Hkv, D = _cache_dims(k_cache, v_cache)
     dev = k_cache.device

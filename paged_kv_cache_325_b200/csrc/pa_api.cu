@@ -265,8 +265,11 @@ pa_status pa_decode_split(void *out, const void *q, const void *k_cache, const v
 
 size_t pa_prefill_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t num_q_heads, int32_t num_kv_heads,
                                  int32_t head_dim) {
-    (void)batch, (void)max_seqlen_q, (void)num_q_heads, (void)num_kv_heads, (void)head_dim;
-    return 0;
+    (void)head_dim;
+    if (batch <= 0 || max_seqlen_q <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+        num_q_heads % num_kv_heads != 0 || 128 % (num_q_heads / num_kv_heads) != 0)
+        return 0;
+    return pa::prefill_workspace_bytes(batch, max_seqlen_q, num_q_heads / num_kv_heads);
 }
 
 pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const void *k_cache, const void *v_cache,
@@ -275,7 +278,6 @@ pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const voi
                             int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                             int32_t num_blocks, int32_t block_size, float softmax_scale, int32_t causal,
                             void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream) {
-    (void)workspace, (void)workspace_bytes;
     if (batch < 0) return fail(PA_ERR_INVALID_ARG, "batch < 0");
     pa_status st = check_cache_shape(num_blocks, block_size, num_kv_heads, head_dim);
     if (st != PA_OK) return st;
@@ -289,8 +291,14 @@ pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const voi
     if (max_seqlen_q < 0 || max_seqlen_k < 1 || max_seqlen_k < max_seqlen_q)
         return fail(PA_ERR_INVALID_ARG, "need 0 <= max_seqlen_q <= max_seqlen_k and max_seqlen_k >= 1");
     if (block_table_stride < 1) return fail(PA_ERR_INVALID_ARG, "block_table_stride must be >= 1");
-    if ((int64_t)max_seqlen_q > (int64_t)65535 * (128 / (num_q_heads / num_kv_heads)))
-        return fail(PA_ERR_UNSUPPORTED, "max_seqlen_q %d is too long for one launch", max_seqlen_q);
+    if (batch > pa::kPrefillMaxBatch) return fail(PA_ERR_UNSUPPORTED, "batch > %d", pa::kPrefillMaxBatch);
+    {
+        const size_t need = pa::prefill_workspace_bytes(batch, max_seqlen_q, num_q_heads / num_kv_heads);
+        if (!workspace || workspace_bytes < need)
+            return fail(PA_ERR_WORKSPACE, "prefill workspace of %zu bytes needed, %zu given", need,
+                        workspace ? workspace_bytes : (size_t)0);
+        if (!aligned(workspace, 256)) return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    }
     if (!out || !q || !k_cache || !v_cache || !cu_seqlens_q || !cu_seqlens_k || !block_table)
         return fail(PA_ERR_INVALID_ARG, "NULL pointer");
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
@@ -318,6 +326,8 @@ pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const voi
     a.max_seqlen_k = max_seqlen_k;
     a.causal = causal ? 1 : 0;
     a.total_q = total_q;
+    a.ranks = (max_seqlen_q + 2 * (128 / a.group) - 1) / (2 * (128 / a.group));
+    a.workspace = workspace;
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
 
     CUtensorMap tm_k, tm_v;

@@ -58,8 +58,12 @@ struct PrefillArgs {
     int32_t *dev_error;
     int32_t bt_stride, batch, num_q_heads, num_kv_heads, group, head_dim;
     int32_t num_blocks, block_size, box_tokens, max_seqlen_q, max_seqlen_k, causal, total_q;
+    int32_t ranks;              // pairs of Q tiles of the longest sequence
+    void *workspace;            // unit table + hand-out counter (prefill_workspace_bytes)
     float scale_log2;
 };
+size_t prefill_workspace_bytes(int32_t batch, int32_t max_seqlen_q, int32_t group);
+constexpr int32_t kPrefillMaxBatch = 6144;   // the planning kernel keeps 2 ints per sequence in shared memory
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                            const CUtensorMap &tm_v, cudaStream_t stream);
 

@@ -50,6 +50,8 @@ constexpr int kMmaWarp = 9;
 constexpr int kThreads = 320;          // 2 softmax warpgroups + TMA warp + MMA warp
 constexpr int kRowBytes = 128;         // one 64-element bf16 swizzle row
 constexpr int kSlab = kM * kRowBytes;  // 128 rows x 128 B = 16 KB
+constexpr int kUnitQueue = 4;          // unit ids handed from the TMA warp to the other roles
+constexpr int kPlanThreads = 1024;
 
 template <int D>
 struct PrefillCfg {
@@ -61,9 +63,9 @@ struct PrefillCfg {
     static constexpr int kPOff = kQOff + 2 * kTileBytes;        // P_A, P_B
     static constexpr int kRingOff = kPOff + 2 * kPBytes;
     static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
-    // kv_full[S] kv_empty[S] q_full q_empty s_full[2] p_full[2] o_full[2] o_empty[2] done
-    static constexpr int kNumBars = 2 * kSlots + 11;
-    static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+    // kv_full[S] kv_empty[S] q_full q_empty s_full[2] p_full[2] o_full[2] o_empty[2] done uq_full[4] uq_empty[4]
+    static constexpr int kNumBars = 2 * kSlots + 11 + 2 * kUnitQueue;
+    static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + kUnitQueue * 4 + 1024;
     static constexpr uint32_t kTmemCols = 512;                  // S_A 0, O_A 128, S_B 256, O_B 384
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -83,38 +85,151 @@ struct Unit {
     int nk;          // key tiles loaded for the unit
 };
 
-// Unit u of the cost-ordered list: rank r = u / (batch * Hkv) counts pairs of
-// Q tiles from the end of each sequence (r = 0: the last, longest pair).
-__device__ __forceinline__ Unit unit_of(const PrefillArgs &a, int u, int TQ) {
+// Geometry of one sequence; false when its cu_seqlens are inconsistent.
+__device__ __forceinline__ bool seq_geometry(const PrefillArgs &a, int s, int &q0, int &n_new, int &n_k) {
+    q0 = a.cu_q[s];
+    const int q1 = a.cu_q[s + 1];
+    const int k0 = a.cu_k[s], k1 = a.cu_k[s + 1];
+    n_new = q1 - q0;
+    n_k = k1 - k0;
+    return !(n_new < 0 || n_k < n_new || q0 < 0 || k0 < 0 || q1 > a.total_q || n_new > a.max_seqlen_q ||
+             n_k > a.max_seqlen_k || (int64_t)n_k > (int64_t)a.bt_stride * a.block_size);
+}
+
+// Work-unit table written by prefill_plan_kernel into the workspace:
+//   [0] counter (next unit to hand out)   [1] total units   [2] R (ranks)
+//   prefix[R + 1] at word 16: units in ranks < r;  order[batch] after it: sequences, longest first.
+// Unit u has rank r (prefix[r] <= u < prefix[r + 1]) = the r-th pair of Q tiles counted from the end of
+// its sequence, and within a rank the sequences come longest first, KV head fastest, so the list runs
+// from the most to the least expensive unit and a greedy hand-out balances the CTAs.
+struct PlanView {
+    unsigned int *counter;
+    const int32_t *prefix, *order;
+    int32_t R, total;
+};
+
+__device__ __forceinline__ PlanView plan_view(void *ws, int32_t R, int32_t batch) {
+    int32_t *w = static_cast<int32_t *>(ws);
+    PlanView v;
+    v.counter = reinterpret_cast<unsigned int *>(w);
+    v.R = R;
+    v.prefix = w + 16;
+    v.order = w + 16 + R + 1;
+    v.total = 0;
+    (void)batch;
+    return v;
+}
+
+__device__ __forceinline__ Unit unit_from_id(const PrefillArgs &a, const PlanView &P, int u, int TQ) {
     Unit U;
     U.valid = false;
-    const int per_rank = a.batch * a.num_kv_heads;
-    const int r = u / per_rank, sk = u % per_rank;
-    U.s = sk / a.num_kv_heads;
-    U.kvh = sk % a.num_kv_heads;
-    const int q0 = __ldg(a.cu_q + U.s), q1 = __ldg(a.cu_q + U.s + 1);
-    const int k0 = __ldg(a.cu_k + U.s), k1 = __ldg(a.cu_k + U.s + 1);
-    U.n_new = q1 - q0;
-    U.n_k = k1 - k0;
-    U.c = U.n_k - U.n_new;
-    if (U.n_new < 0 || U.c < 0 || q0 < 0 || k0 < 0 || q1 > a.total_q || U.n_new > a.max_seqlen_q ||
-        U.n_k > a.max_seqlen_k || (int64_t)U.n_k > (int64_t)a.bt_stride * a.block_size) {
-        if (r == 0 && U.kvh == 0 && threadIdx.x == 0) report(a.dev_error, PA_DEVERR_SEQLENS);
-        return U;
+    int lo = 0, hi = P.R;                         // prefix[lo] <= u < prefix[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (P.prefix[mid] <= u) lo = mid; else hi = mid;
     }
-    const int npairs = (U.n_new + 2 * TQ - 1) / (2 * TQ);
+    const int r = lo, i = u - P.prefix[r];
+    U.s = P.order[i / a.num_kv_heads];
+    U.kvh = i % a.num_kv_heads;
+    int q0, n_new, n_k;
+    if (!seq_geometry(a, U.s, q0, n_new, n_k)) return U;
+    U.n_new = n_new;
+    U.n_k = n_k;
+    U.c = n_k - n_new;
+    const int npairs = (n_new + 2 * TQ - 1) / (2 * TQ);
     if (r >= npairs) return U;
     const int p = npairs - 1 - r;
     U.q0 = q0;
     for (int x = 0; x < 2; ++x) {
         U.tok0[x] = (2 * p + x) * TQ;
-        U.nq[x] = max(0, min(TQ, U.n_new - U.tok0[x]));
-        U.kend[x] = U.nq[x] == 0 ? 0 : (a.causal ? U.c + U.tok0[x] + U.nq[x] : U.n_k);
+        U.nq[x] = max(0, min(TQ, n_new - U.tok0[x]));
+        U.kend[x] = U.nq[x] == 0 ? 0 : (a.causal ? U.c + U.tok0[x] + U.nq[x] : n_k);
         U.nt[x] = (U.kend[x] + kN - 1) / kN;
     }
     U.nk = max(U.nt[0], U.nt[1]);
     U.valid = true;
     return U;
+}
+
+// One CTA: validate every sequence, sort the sequences by their number of Q-tile pairs (longest first),
+// count the units of every rank, write the prefix sums and zero the hand-out counter.
+__global__ void __launch_bounds__(kPlanThreads)
+    prefill_plan_kernel(const PrefillArgs a, int32_t R, int32_t two_tq) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the main kernel may start its prologue
+    extern __shared__ int32_t plan_smem[];
+    int32_t *np = plan_smem;                  // [batch] pairs per sequence
+    int32_t *nps = plan_smem + a.batch;       // [batch] pairs, sorted descending
+    __shared__ int32_t warp_tot[32];
+    int32_t *w = static_cast<int32_t *>(a.workspace);
+    int32_t *prefix = w + 16;
+    int32_t *order = w + 16 + R + 1;
+    const int tid = threadIdx.x;
+    for (int s = tid; s < a.batch; s += kPlanThreads) {
+        int q0, n_new, n_k;
+        if (seq_geometry(a, s, q0, n_new, n_k)) {
+            np[s] = min(R, (n_new + two_tq - 1) / two_tq);
+        } else {
+            np[s] = 0;
+            report(a.dev_error, PA_DEVERR_SEQLENS);
+        }
+    }
+    __syncthreads();
+    for (int s = tid; s < a.batch; s += kPlanThreads) {
+        const int v = np[s];
+        int rank = 0;
+        for (int t = 0; t < a.batch; ++t) rank += (np[t] > v) || (np[t] == v && t < s);
+        order[rank] = s;
+        nps[rank] = v;
+    }
+    __syncthreads();
+    // units of rank r = Hkv * #{s : np[s] > r}; nps is descending, so count by binary search
+    const int chunk = (R + kPlanThreads - 1) / kPlanThreads;
+    const int r0 = min(R, tid * chunk), r1 = min(R, r0 + chunk);
+    int32_t local = 0;
+    for (int r = r0; r < r1; ++r) {
+        int lo = 0, hi = a.batch;                 // first index with nps <= r
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (nps[mid] > r) lo = mid + 1; else hi = mid;
+        }
+        local += lo * a.num_kv_heads;
+    }
+    // exclusive block scan of `local`
+    const int lane = tid & 31, wid = tid >> 5;
+    int32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int32_t t = warp_tot[lane], ti = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, ti, o);
+            if (lane >= o) ti += y;
+        }
+        warp_tot[lane] = ti - t;                  // exclusive prefix of the warp totals
+    }
+    __syncthreads();
+    int32_t run = warp_tot[wid] + incl - local;
+    for (int r = r0; r < r1; ++r) {
+        prefix[r] = run;
+        int lo = 0, hi = a.batch;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (nps[mid] > r) lo = mid + 1; else hi = mid;
+        }
+        run += lo * a.num_kv_heads;
+    }
+    if (r1 == R && r0 < R) prefix[R] = run;
+    if (R == 0 && tid == 0) prefix[0] = 0;
+    if (tid == 0) {
+        w[0] = 0;                                 // hand-out counter
+        w[2] = R;
+    }
 }
 
 template <int D>
@@ -134,13 +249,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *o_full = p_full + 2;     // [2]
     uint64_t *o_empty = o_full + 2;    // [2]
     uint64_t *done = o_empty + 2;
+    uint64_t *uq_full = done + 1;      // [kUnitQueue]
+    uint64_t *uq_empty = uq_full + kUnitQueue;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
+    volatile int32_t *unit_q = reinterpret_cast<volatile int32_t *>(tmem_slot + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.group;
     const int TQ = kM / G;
-    const int per_rank = a.batch * a.num_kv_heads;
-    const int num_units = ((a.max_seqlen_q + 2 * TQ - 1) / (2 * TQ)) * per_rank;
+    const PlanView plan = plan_view(a.workspace, a.ranks, a.batch);
 
     const uint32_t sbase = smem_u32(smem);
     const uint32_t q_s = sbase + C::kQOff;
@@ -161,6 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(o_empty + x), 4);
         }
         mbar_init(smem_u32(done), 1);
+        for (int i = 0; i < kUnitQueue; ++i) {
+            mbar_init(smem_u32(uq_full + i), 1);
+            mbar_init(smem_u32(uq_empty + i), 9);   // the MMA warp and the eight softmax warps
+        }
         fence_barrier_init();
     }
     if (warp == kMmaWarp) {
@@ -171,6 +292,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // everything above overlapped the planning kernel; its table (and all earlier work) is visible after this
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    // unit hand-out: the TMA warp pushes unit ids (-1 ends the stream); the other roles pop them in order
+    auto pop_unit = [&](uint32_t k, bool arrive) -> int {
+        const int slot = k % kUnitQueue;
+        if (!mbar_wait(smem_u32(uq_full + slot), (k / kUnitQueue) & 1, a.dev_error)) return -1;
+        const int u = unit_q[slot];
+        __syncwarp();
+        if (arrive) mbar_arrive(smem_u32(uq_empty + slot));
+        return u;
+    };
 
     if (warp == kTmaWarp) {
         // ============================================================ TMA ==
@@ -179,10 +312,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             const int B = a.block_size, box = a.box_tokens;
-            uint32_t nq = 0, L = 0;
+            uint32_t nq = 0, L = 0, nu = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
-                const Unit U = unit_of(a, u, TQ);
+            const int total = plan.prefix[plan.R];
+            for (;; ++nu) {
+                int u = ok ? (int)atomicAdd(plan.counter, 1u) : -1;
+                if (u >= total) u = -1;
+                const int slot = nu % kUnitQueue;
+                if (nu >= (uint32_t)kUnitQueue &&
+                    !mbar_wait(smem_u32(uq_empty + slot), (nu / kUnitQueue - 1) & 1, a.dev_error))
+                    u = -1;
+                unit_q[slot] = u;
+                mbar_arrive(smem_u32(uq_full + slot));
+                if (u < 0) break;
+                const Unit U = unit_from_id(a, plan, u, TQ);
                 if (!U.valid) continue;
                 if (nq > 0 && !mbar_wait(smem_u32(q_empty), (nq - 1) & 1, a.dev_error)) break;
                 mbar_arrive_expect_tx(smem_u32(q_full), (uint32_t)(2 * C::kTileBytes));
@@ -266,8 +409,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) tc_commit(smem_u32(bar));
             __syncwarp();
         };
-        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
-            const Unit U = unit_of(a, u, TQ);
+        for (uint32_t k = 0; ok; ++k) {
+            const int u = pop_unit(k, lane == 0);
+            if (u < 0) break;
+            const Unit U = unit_from_id(a, plan, u, TQ);
             if (!U.valid) continue;
             if (!mbar_wait(smem_u32(q_full), nq & 1, a.dev_error)) break;
             ++nq;
@@ -340,8 +485,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const float sl = a.scale_log2;
         uint32_t ns = 0, no = 0;
-        for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
-            const Unit U = unit_of(a, u, TQ);
+        for (uint32_t k = 0;; ++k) {
+            const int u = pop_unit(k, lane == 0);
+            if (u < 0) break;
+            const Unit U = unit_from_id(a, plan, u, TQ);
             if (!U.valid || U.nt[x] == 0) continue;
             const int t = U.tok0[x] + r / G;              // this row's new-token index
             int lim = a.causal ? U.c + t : U.n_k - 1;      // last visible key
@@ -479,14 +626,34 @@ cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &tm_q, cons
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
     const int TQ = kM / a.group;
-    const int64_t units = (int64_t)((a.max_seqlen_q + 2 * TQ - 1) / (2 * TQ)) * a.batch * a.num_kv_heads;
-    const int grid = (int)(units < num_sms() ? units : num_sms());
+    const size_t plan_smem = (size_t)2 * a.batch * sizeof(int32_t);
+    prefill_plan_kernel<<<1, kPlanThreads, plan_smem, stream>>>(a, a.ranks, 2 * TQ);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t max_units = (int64_t)a.ranks * a.batch * a.num_kv_heads;
+    const int grid = (int)(max_units < num_sms() ? max_units : num_sms());
     if (grid <= 0) return cudaSuccess;
-    prefill_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tm_q, tm_k, tm_v, a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<D>, tm_q, tm_k, tm_v, a);
 }
 
 }  // namespace
+
+size_t prefill_workspace_bytes(int32_t batch, int32_t max_seqlen_q, int32_t group) {
+    const int32_t TQ = kM / group;
+    const int64_t R = ((int64_t)max_seqlen_q + 2 * TQ - 1) / (2 * TQ);
+    const size_t words = 16 + (size_t)(R + 1) + (size_t)batch;
+    return (words * sizeof(int32_t) + 255) / 256 * 256;
+}
 
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                            const CUtensorMap &tm_v, cudaStream_t stream) {

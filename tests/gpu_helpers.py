@@ -85,6 +85,7 @@ class PrefillOnGpu:
         self.cu_q = i32(case.cu_seqlens_q, self.dev)
         self.cu_k = i32(case.cu_seqlens_k, self.dev)
         self.out = torch.empty_like(self.q)
+        self.ws = pa.alloc_prefill_workspace(self.q, case.num_kv_heads, case.batch, max(1, case.max_seqlen_q))
 
     def store(self, dev_error=None):
         pa.pa_store_kv(self.k_new, self.v_new, self.slot_mapping, self.k_cache, self.v_cache, dev_error=dev_error)
@@ -93,7 +94,7 @@ class PrefillOnGpu:
         c = self.case
         pa.pa_prefill_varlen(self.out, self.q, self.k_cache, self.v_cache, self.cu_q, self.cu_k, c.max_seqlen_q,
                              c.max_seqlen_k, self.block_table, c.softmax_scale,
-                             causal=c.causal if causal is None else causal, dev_error=dev_error)
+                             causal=c.causal if causal is None else causal, workspace=self.ws, dev_error=dev_error)
         return self.out
 
 

@@ -98,11 +98,11 @@ def test_decode_workspace_size_query():
 
 def _prefill(lib, **kw):
     a = dict(out=A, q=A, tq=150, kc=A, vc=A, cq=A, ck=A, mq=100, mk=200, bt=A, bts=4, batch=2, Hq=32, Hkv=8, D=128,
-             nb=16, B=256, scale=0.088, causal=1, err=None)
+             nb=16, B=256, scale=0.088, causal=1, err=None, ws=A, wsb=1 << 20)
     a.update(kw)
-    return lib.pa_prefill_varlen(a["out"], a["q"], a["tq"], a["kc"], a["vc"], a["cq"], a["ck"], a["mq"], a["mk"], a["bt"],
-                                 a["bts"], a["batch"], a["Hq"], a["Hkv"], a["D"], a["nb"], a["B"], a["scale"],
-                                 a["causal"], None, 0, a["err"], None)
+    return lib.pa_prefill_varlen(a["out"], a["q"], a["tq"], a["kc"], a["vc"], a["cq"], a["ck"], a["mq"], a["mk"],
+                                 a["bt"], a["bts"], a["batch"], a["Hq"], a["Hkv"], a["D"], a["nb"], a["B"],
+                                 a["scale"], a["causal"], a["ws"], a["wsb"], a["err"], None)
 
 
 def test_prefill_validation(lib):
@@ -115,6 +115,11 @@ def test_prefill_validation(lib):
     assert _prefill(lib, mq=0) == pa.PA_OK
     assert _prefill(lib, tq=0) == pa.PA_OK
     assert _prefill(lib, tq=-1) == pa.PA_ERR_INVALID_ARG
+    assert _prefill(lib, ws=None, wsb=0) == pa.PA_ERR_WORKSPACE     # no workspace for the unit table
+    need = pa.pa_prefill_workspace_size(2, 100, 32, 8, 128)
+    assert need >= 4 * (16 + 2 + 1 + 2)
+    assert _prefill(lib, ws=A, wsb=need - 1) == pa.PA_ERR_WORKSPACE
+    assert _prefill(lib, batch=7000, ws=A, wsb=1 << 20) == pa.PA_ERR_UNSUPPORTED
 
 
 def test_selftest_validation(lib):

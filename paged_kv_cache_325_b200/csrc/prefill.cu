@@ -65,7 +65,7 @@ struct PrefillCfg {
     static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
     // kv_full[S] kv_empty[S] q_full q_empty s_full[2] p_full[2] o_full[2] o_empty[2] done uq_full[4] uq_empty[4]
     static constexpr int kNumBars = 2 * kSlots + 11 + 2 * kUnitQueue;
-    static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + kUnitQueue * 4 + 1024;
+    static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 64 + kUnitQueue * 64 + 1024;
     static constexpr uint32_t kTmemCols = 512;                  // S_A 0, O_A 128, S_B 256, O_B 384
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -73,8 +73,8 @@ struct PrefillCfg {
 __device__ __forceinline__ uint32_t col_s(int x) { return x ? 256u : 0u; }
 __device__ __forceinline__ uint32_t col_o(int x) { return x ? 384u : 128u; }
 
-struct Unit {
-    bool valid;
+struct Unit {                 // 16 words; copied through the shared-memory unit queue
+    int valid;
     int s, kvh;
     int q0;          // row of the sequence's first new token in q / out
     int n_new, n_k, c;
@@ -84,6 +84,7 @@ struct Unit {
     int nt[2];       // key tiles of tile A / B
     int nk;          // key tiles loaded for the unit
 };
+static_assert(sizeof(Unit) == 64, "Unit is copied as 16 words");
 
 // Geometry of one sequence; false when its cu_seqlens are inconsistent.
 __device__ __forceinline__ bool seq_geometry(const PrefillArgs &a, int s, int &q0, int &n_new, int &n_k) {
@@ -122,7 +123,7 @@ __device__ __forceinline__ PlanView plan_view(void *ws, int32_t R, int32_t batch
 
 __device__ __forceinline__ Unit unit_from_id(const PrefillArgs &a, const PlanView &P, int u, int TQ) {
     Unit U;
-    U.valid = false;
+    U.valid = 0;
     int lo = 0, hi = P.R;                         // prefix[lo] <= u < prefix[hi]
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -147,7 +148,7 @@ __device__ __forceinline__ Unit unit_from_id(const PrefillArgs &a, const PlanVie
         U.nt[x] = (U.kend[x] + kN - 1) / kN;
     }
     U.nk = max(U.nt[0], U.nt[1]);
-    U.valid = true;
+    U.valid = 1;
     return U;
 }
 
@@ -252,7 +253,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *uq_full = done + 1;      // [kUnitQueue]
     uint64_t *uq_empty = uq_full + kUnitQueue;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
-    volatile int32_t *unit_q = reinterpret_cast<volatile int32_t *>(tmem_slot + 4);
+    // unit queue: kUnitQueue entries of 16 words (a decoded Unit; valid = -1 ends the stream)
+    volatile int32_t *unit_q = reinterpret_cast<volatile int32_t *>(tmem_slot + 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.group;
@@ -295,14 +297,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // everything above overlapped the planning kernel; its table (and all earlier work) is visible after this
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // unit hand-out: the TMA warp pushes unit ids (-1 ends the stream); the other roles pop them in order
-    auto pop_unit = [&](uint32_t k, bool arrive) -> int {
+    // unit hand-out: the TMA warp fetches unit ids, decodes them once and pushes the decoded units
+    // (valid = -1 ends the stream); the other roles pop them in order
+    auto pop_unit = [&](uint32_t k, bool arrive, Unit &U) -> bool {
         const int slot = k % kUnitQueue;
-        if (!mbar_wait(smem_u32(uq_full + slot), (k / kUnitQueue) & 1, a.dev_error)) return -1;
-        const int u = unit_q[slot];
+        if (!mbar_wait(smem_u32(uq_full + slot), (k / kUnitQueue) & 1, a.dev_error)) return false;
+        int32_t *dst = reinterpret_cast<int32_t *>(&U);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dst[i] = unit_q[slot * 16 + i];
         __syncwarp();
         if (arrive) mbar_arrive(smem_u32(uq_empty + slot));
-        return u;
+        return U.valid >= 0;
     };
 
     if (warp == kTmaWarp) {
@@ -318,14 +323,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (;; ++nu) {
                 int u = ok ? (int)atomicAdd(plan.counter, 1u) : -1;
                 if (u >= total) u = -1;
+                Unit U;
+                if (u >= 0) U = unit_from_id(a, plan, u, TQ);
+                else U.valid = -1;
                 const int slot = nu % kUnitQueue;
                 if (nu >= (uint32_t)kUnitQueue &&
                     !mbar_wait(smem_u32(uq_empty + slot), (nu / kUnitQueue - 1) & 1, a.dev_error))
-                    u = -1;
-                unit_q[slot] = u;
+                    U.valid = -1;
+                const int32_t *src = reinterpret_cast<const int32_t *>(&U);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) unit_q[slot * 16 + i] = src[i];
                 mbar_arrive(smem_u32(uq_full + slot));
-                if (u < 0) break;
-                const Unit U = unit_from_id(a, plan, u, TQ);
+                if (U.valid < 0) break;
                 if (!U.valid) continue;
                 if (nq > 0 && !mbar_wait(smem_u32(q_empty), (nq - 1) & 1, a.dev_error)) break;
                 mbar_arrive_expect_tx(smem_u32(q_full), (uint32_t)(2 * C::kTileBytes));
@@ -410,9 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
         };
         for (uint32_t k = 0; ok; ++k) {
-            const int u = pop_unit(k, lane == 0);
-            if (u < 0) break;
-            const Unit U = unit_from_id(a, plan, u, TQ);
+            Unit U;
+            if (!pop_unit(k, lane == 0, U)) break;
             if (!U.valid) continue;
             if (!mbar_wait(smem_u32(q_full), nq & 1, a.dev_error)) break;
             ++nq;
@@ -486,9 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sl = a.scale_log2;
         uint32_t ns = 0, no = 0;
         for (uint32_t k = 0;; ++k) {
-            const int u = pop_unit(k, lane == 0);
-            if (u < 0) break;
-            const Unit U = unit_from_id(a, plan, u, TQ);
+            Unit U;
+            if (!pop_unit(k, lane == 0, U)) break;
             if (!U.valid || U.nt[x] == 0) continue;
             const int t = U.tok0[x] + r / G;              // this row's new-token index
             int lim = a.causal ? U.c + t : U.n_k - 1;      // last visible key
@@ -573,22 +580,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) +
                                                    ((int64_t)(U.q0 + (store ? t : 0)) * a.num_q_heads +
                                                     (int64_t)U.kvh * G + r % G) * D);
+            uint32_t o[D / 32][32];
 #pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
-                uint32_t o[32];
-                tmem_ld32(lane_base + col_o(x) + q * 32, o);
-                tc_wait_ld();
-                if (store) {
+            for (int q = 0; q < D / 32; ++q) tmem_ld32(lane_base + col_o(x) + q * 32, o[q]);
+            tc_wait_ld();
+            if (store) {
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q)
 #pragma unroll
                     for (int e = 0; e < 32; e += 8) {
                         uint4 v;
-                        v.x = pack_bf16(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
-                        v.y = pack_bf16(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-                        v.z = pack_bf16(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
-                        v.w = pack_bf16(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+                        v.x = pack_bf16(__uint_as_float(o[q][e]) * inv, __uint_as_float(o[q][e + 1]) * inv);
+                        v.y = pack_bf16(__uint_as_float(o[q][e + 2]) * inv, __uint_as_float(o[q][e + 3]) * inv);
+                        v.z = pack_bf16(__uint_as_float(o[q][e + 4]) * inv, __uint_as_float(o[q][e + 5]) * inv);
+                        v.w = pack_bf16(__uint_as_float(o[q][e + 6]) * inv, __uint_as_float(o[q][e + 7]) * inv);
                         dst[(q * 32 + e) / 8] = v;
                     }
-                }
             }
             tc_fence_before();
             __syncwarp();

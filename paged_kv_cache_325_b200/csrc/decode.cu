@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             tma_prefetch_desc(&tm_v);
             const int32_t *bt = a.block_table + (int64_t)s * a.bt_stride;
             const int B = a.block_size, box = a.box_tokens;
+            int issued = 0;
             for (int i = 0; i < ntiles; ++i) {
                 const int st = i % C::kStages;
                 if (i >= C::kStages && !mbar_wait(smem_u32(empty + st), ((i / C::kStages) & 1) ^ 1, a.dev_error))
@@ -124,7 +125,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                         tma_load_3d(vdst + off, &tm_v, h * 64, kvh, row, fb);
                     }
                 }
+                issued = i + 1;
             }
+            // leave no TMA copy in flight: wait (bounded) for the last load of every stage; on the normal path
+            // the consumers have already waited for them all and these return at once
+            for (int i = (issued > C::kStages ? issued - C::kStages : 0); i < issued; ++i)
+                mbar_wait(smem_u32(full + i % C::kStages), (i / C::kStages) & 1, a.dev_error);
         }
         return;
     }

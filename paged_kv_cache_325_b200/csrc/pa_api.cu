@@ -269,7 +269,7 @@ size_t pa_prefill_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t nu
     if (batch <= 0 || max_seqlen_q <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
         num_q_heads % num_kv_heads != 0 || 128 % (num_q_heads / num_kv_heads) != 0)
         return 0;
-    return pa::prefill_workspace_bytes(batch, max_seqlen_q, num_q_heads / num_kv_heads);
+    return pa::prefill_workspace_bytes(batch, max_seqlen_q, num_q_heads / num_kv_heads, num_kv_heads);
 }
 
 pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const void *k_cache, const void *v_cache,
@@ -293,7 +293,7 @@ pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const voi
     if (block_table_stride < 1) return fail(PA_ERR_INVALID_ARG, "block_table_stride must be >= 1");
     if (batch > pa::kPrefillMaxBatch) return fail(PA_ERR_UNSUPPORTED, "batch > %d", pa::kPrefillMaxBatch);
     {
-        const size_t need = pa::prefill_workspace_bytes(batch, max_seqlen_q, num_q_heads / num_kv_heads);
+        const size_t need = pa::prefill_workspace_bytes(batch, max_seqlen_q, num_q_heads / num_kv_heads, num_kv_heads);
         if (!workspace || workspace_bytes < need)
             return fail(PA_ERR_WORKSPACE, "prefill workspace of %zu bytes needed, %zu given", need,
                         workspace ? workspace_bytes : (size_t)0);

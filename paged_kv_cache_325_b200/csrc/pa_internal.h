@@ -62,7 +62,7 @@ struct PrefillArgs {
     void *workspace;            // unit table + hand-out counter (prefill_workspace_bytes)
     float scale_log2;
 };
-size_t prefill_workspace_bytes(int32_t batch, int32_t max_seqlen_q, int32_t group);
+size_t prefill_workspace_bytes(int32_t batch, int32_t max_seqlen_q, int32_t group, int32_t num_kv_heads);
 constexpr int32_t kPrefillMaxBatch = 6144;   // the planning kernel keeps 2 ints per sequence in shared memory
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                            const CUtensorMap &tm_v, cudaStream_t stream);

@@ -56,17 +56,16 @@ constexpr int kPlanThreads = 1024;
 template <int D>
 struct PrefillCfg {
     static constexpr int kHalves = D / 64;
-    static constexpr int kSlots = D == 128 ? 3 : 6;             // K/V ring slots (one K or V tile each)
+    static constexpr int kSlots = D == 128 ? 5 : 8;             // K/V ring slots (one K or V tile each)
     static constexpr int kTileBytes = kHalves * kSlab;          // a Q tile, or a K or V tile of 128 keys
-    static constexpr int kPBytes = 2 * kSlab;                   // P: 128 rows x 128 keys bf16
     static constexpr int kQOff = 0;                             // Q_A, Q_B
-    static constexpr int kPOff = kQOff + 2 * kTileBytes;        // P_A, P_B
-    static constexpr int kRingOff = kPOff + 2 * kPBytes;
+    static constexpr int kRingOff = kQOff + 2 * kTileBytes;
     static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
     // kv_full[S] kv_empty[S] q_full q_empty s_full[2] p_full[2] o_full[2] o_empty[2] done uq_full[4] uq_empty[4]
     static constexpr int kNumBars = 2 * kSlots + 11 + 2 * kUnitQueue;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 64 + kUnitQueue * 64 + 1024;
     static constexpr uint32_t kTmemCols = 512;                  // S_A 0, O_A 128, S_B 256, O_B 384
+                                                                // (P_X, bf16, overwrites the first 64 columns of S_X)
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -97,54 +96,46 @@ __device__ __forceinline__ bool seq_geometry(const PrefillArgs &a, int s, int &q
              n_k > a.max_seqlen_k || (int64_t)n_k > (int64_t)a.bt_stride * a.block_size);
 }
 
-// Work-unit table written by prefill_plan_kernel into the workspace:
-//   [0] counter (next unit to hand out)   [1] total units   [2] R (ranks)
-//   prefix[R + 1] at word 16: units in ranks < r;  order[batch] after it: sequences, longest first.
-// Unit u has rank r (prefix[r] <= u < prefix[r + 1]) = the r-th pair of Q tiles counted from the end of
-// its sequence, and within a rank the sequences come longest first, KV head fastest, so the list runs
-// from the most to the least expensive unit and a greedy hand-out balances the CTAs.
-struct PlanView {
-    unsigned int *counter;
-    const int32_t *prefix, *order;
-    int32_t R, total;
+// Work-unit table written by prefill_plan_kernel into the workspace (int32 words):
+//   w[0] hand-out counter, w[1] number of units, w[2] R (ranks)
+//   prefix[R + 1] at word 16: units in ranks < r
+//   order[batch]: sequences, longest first
+//   geo[batch] (int4, 16-byte aligned): q0, n_new, n_k, valid of every sequence
+//   units[R * batch * Hkv] (int4): s, kv head, rank of every unit, in hand-out order
+// Unit u has rank r = the r-th pair of Q tiles counted from the end of its sequence; ranks come in
+// increasing order and, within a rank, sequences longest first, so the list runs from the most to the
+// least expensive unit and a greedy hand-out balances the CTAs.
+struct PlanLayout {
+    int32_t prefix, order, geo, units;   // word offsets
 };
 
-__device__ __forceinline__ PlanView plan_view(void *ws, int32_t R, int32_t batch) {
-    int32_t *w = static_cast<int32_t *>(ws);
-    PlanView v;
-    v.counter = reinterpret_cast<unsigned int *>(w);
-    v.R = R;
-    v.prefix = w + 16;
-    v.order = w + 16 + R + 1;
-    v.total = 0;
-    (void)batch;
-    return v;
+__host__ __device__ __forceinline__ PlanLayout plan_layout(int32_t R, int32_t batch) {
+    PlanLayout l;
+    l.prefix = 16;
+    l.order = l.prefix + R + 1;
+    l.geo = (l.order + batch + 3) & ~3;
+    l.units = l.geo + 4 * batch;
+    return l;
 }
 
-__device__ __forceinline__ Unit unit_from_id(const PrefillArgs &a, const PlanView &P, int u, int TQ) {
+__device__ __forceinline__ Unit unit_from_record(const PrefillArgs &a, int4 rec, int4 geo, int TQ) {
     Unit U;
     U.valid = 0;
-    int lo = 0, hi = P.R;                         // prefix[lo] <= u < prefix[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (P.prefix[mid] <= u) lo = mid; else hi = mid;
-    }
-    const int r = lo, i = u - P.prefix[r];
-    U.s = P.order[i / a.num_kv_heads];
-    U.kvh = i % a.num_kv_heads;
-    int q0, n_new, n_k;
-    if (!seq_geometry(a, U.s, q0, n_new, n_k)) return U;
-    U.n_new = n_new;
-    U.n_k = n_k;
-    U.c = n_k - n_new;
-    const int npairs = (n_new + 2 * TQ - 1) / (2 * TQ);
+    U.s = rec.x;
+    U.kvh = rec.y;
+    const int r = rec.z;
+    if (!geo.w) return U;
+    U.q0 = geo.x;
+    U.n_new = geo.y;
+    U.n_k = geo.z;
+    U.c = U.n_k - U.n_new;
+    const int npairs = (U.n_new + 2 * TQ - 1) / (2 * TQ);
     if (r >= npairs) return U;
     const int p = npairs - 1 - r;
-    U.q0 = q0;
     for (int x = 0; x < 2; ++x) {
         U.tok0[x] = (2 * p + x) * TQ;
-        U.nq[x] = max(0, min(TQ, n_new - U.tok0[x]));
-        U.kend[x] = U.nq[x] == 0 ? 0 : (a.causal ? U.c + U.tok0[x] + U.nq[x] : n_k);
+        U.nq[x] = max(0, min(TQ, U.n_new - U.tok0[x]));
+        U.kend[x] = U.nq[x] == 0 ? 0 : (a.causal ? U.c + U.tok0[x] + U.nq[x] : U.n_k);
         U.nt[x] = (U.kend[x] + kN - 1) / kN;
     }
     U.nk = max(U.nt[0], U.nt[1]);
@@ -162,15 +153,20 @@ __global__ void __launch_bounds__(kPlanThreads)
     int32_t *nps = plan_smem + a.batch;       // [batch] pairs, sorted descending
     __shared__ int32_t warp_tot[32];
     int32_t *w = static_cast<int32_t *>(a.workspace);
-    int32_t *prefix = w + 16;
-    int32_t *order = w + 16 + R + 1;
+    const PlanLayout lay = plan_layout(R, a.batch);
+    int32_t *prefix = w + lay.prefix;
+    int32_t *order = w + lay.order;
+    int4 *geo = reinterpret_cast<int4 *>(w + lay.geo);
+    int4 *units = reinterpret_cast<int4 *>(w + lay.units);
     const int tid = threadIdx.x;
     for (int s = tid; s < a.batch; s += kPlanThreads) {
         int q0, n_new, n_k;
         if (seq_geometry(a, s, q0, n_new, n_k)) {
             np[s] = min(R, (n_new + two_tq - 1) / two_tq);
+            geo[s] = make_int4(q0, n_new, n_k, 1);
         } else {
             np[s] = 0;
+            geo[s] = make_int4(0, 0, 0, 0);
             report(a.dev_error, PA_DEVERR_SEQLENS);
         }
     }
@@ -227,8 +223,20 @@ __global__ void __launch_bounds__(kPlanThreads)
     }
     if (r1 == R && r0 < R) prefix[R] = run;
     if (R == 0 && tid == 0) prefix[0] = 0;
+    __syncthreads();                              // prefix and order are visible to the whole CTA
+    const int total = prefix[R];
+    for (int u = tid; u < total; u += kPlanThreads) {
+        int lo = 0, hi = R;                       // prefix[lo] <= u < prefix[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (prefix[mid] <= u) lo = mid; else hi = mid;
+        }
+        const int i = u - prefix[lo];
+        units[u] = make_int4(order[i / a.num_kv_heads], i % a.num_kv_heads, lo, 0);
+    }
     if (tid == 0) {
         w[0] = 0;                                 // hand-out counter
+        w[1] = total;
         w[2] = R;
     }
 }
@@ -259,11 +267,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.group;
     const int TQ = kM / G;
-    const PlanView plan = plan_view(a.workspace, a.ranks, a.batch);
+    int32_t *plan_w = static_cast<int32_t *>(a.workspace);
+    const PlanLayout plan = plan_layout(a.ranks, a.batch);
 
     const uint32_t sbase = smem_u32(smem);
     const uint32_t q_s = sbase + C::kQOff;
-    const uint32_t p_s = sbase + C::kPOff;
     const uint32_t ring = sbase + C::kRingOff;
 
     if (threadIdx.x == 0) {
@@ -312,72 +320,110 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kTmaWarp) {
         // ============================================================ TMA ==
+        // The whole warp runs this role: every lane waits on the barriers, lane 0 issues the copies, and
+        // block ids are read 32 at a time (one per lane) and passed around with shuffles.
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            const int B = a.block_size, box = a.box_tokens;
-            uint32_t nq = 0, L = 0, nu = 0;
-            bool ok = true;
-            const int total = plan.prefix[plan.R];
-            for (;; ++nu) {
-                int u = ok ? (int)atomicAdd(plan.counter, 1u) : -1;
-                if (u >= total) u = -1;
-                Unit U;
-                if (u >= 0) U = unit_from_id(a, plan, u, TQ);
-                else U.valid = -1;
-                const int slot = nu % kUnitQueue;
-                if (nu >= (uint32_t)kUnitQueue &&
-                    !mbar_wait(smem_u32(uq_empty + slot), (nu / kUnitQueue - 1) & 1, a.dev_error))
-                    U.valid = -1;
+        }
+        const int B = a.block_size, box = a.box_tokens;
+        const int total = plan_w[1];
+        const int4 *units = reinterpret_cast<const int4 *>(plan_w + plan.units);
+        const int4 *geo = reinterpret_cast<const int4 *>(plan_w + plan.geo);
+        auto fetch = [&]() -> int {
+            int u = 0;
+            if (lane == 0) u = (int)atomicAdd(reinterpret_cast<unsigned int *>(plan_w), 1u);
+            return __shfl_sync(0xffffffffu, u, 0);
+        };
+        auto decode = [&](int u) -> Unit {
+            Unit V;
+            if (u >= total) {
+                V.valid = -1;
+                return V;
+            }
+            const int4 rec = units[u];
+            return unit_from_record(a, rec, geo[rec.x], TQ);
+        };
+        uint32_t nq = 0, L = 0;
+        bool ok = true;
+        Unit next = decode(fetch());
+        for (uint32_t nu = 0;; ++nu) {
+            Unit U = next;
+            if (!ok) U.valid = -1;
+            const int slot = nu % kUnitQueue;
+            if (nu >= (uint32_t)kUnitQueue &&
+                !mbar_wait(smem_u32(uq_empty + slot), (nu / kUnitQueue - 1) & 1, a.dev_error))
+                U.valid = -1;
+            if (lane == 0) {
                 const int32_t *src = reinterpret_cast<const int32_t *>(&U);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) unit_q[slot * 16 + i] = src[i];
                 mbar_arrive(smem_u32(uq_full + slot));
-                if (U.valid < 0) break;
-                if (!U.valid) continue;
-                if (nq > 0 && !mbar_wait(smem_u32(q_empty), (nq - 1) & 1, a.dev_error)) break;
-                mbar_arrive_expect_tx(smem_u32(q_full), (uint32_t)(2 * C::kTileBytes));
-                for (int x = 0; x < 2; ++x)
+            }
+            __syncwarp();
+            if (U.valid < 0) break;
+            // take the next unit now; its id and record loads overlap this unit's copies
+            const int next_u = fetch();
+            if (U.valid) {
+                if (nq > 0 && !mbar_wait(smem_u32(q_empty), (nq - 1) & 1, a.dev_error)) ok = false;
+                if (ok && lane == 0) {
+                    mbar_arrive_expect_tx(smem_u32(q_full), (uint32_t)(2 * C::kTileBytes));
+                    for (int x = 0; x < 2; ++x)
 #pragma unroll
-                    for (int h = 0; h < C::kHalves; ++h)
-                        tma_load_3d(q_s + x * C::kTileBytes + h * kSlab, &tm_q, h * 64, U.kvh * G,
-                                    U.q0 + U.tok0[x], smem_u32(q_full));
-                ++nq;
+                        for (int h = 0; h < C::kHalves; ++h)
+                            tma_load_3d(q_s + x * C::kTileBytes + h * kSlab, &tm_q, h * 64, U.kvh * G,
+                                        U.q0 + U.tok0[x], smem_u32(q_full));
+                }
+                if (ok) ++nq;
                 const int32_t *bt = a.block_table + (int64_t)U.s * a.bt_stride;
                 const int kend = max(U.kend[0], U.kend[1]);
+                int chunk = -32, ids = 0;            // block_table[chunk + lane] lives in `ids` of that lane
                 for (int j = 0; j < U.nk && ok; ++j) {
                     const int key0 = j * kN;
                     const int nbox = (min(kN, kend - key0) + box - 1) / box;
-                    for (int kv = 0; kv < 2; ++kv, ++L) {
-                        const int slot = L % C::kSlots;
+                    const int last_blk = (key0 + (nbox - 1) * box) / B;
+                    if (last_blk >= chunk + 32) {
+                        chunk = key0 / B;
+                        ids = chunk + lane < a.bt_stride ? bt[chunk + lane] : -1;
+                    }
+                    for (int kv = 0; kv < 2 && ok; ++kv, ++L) {
+                        const int slot2 = L % C::kSlots;
                         if (L >= (uint32_t)C::kSlots &&
-                            !mbar_wait(smem_u32(kv_empty + slot), (L / C::kSlots - 1) & 1, a.dev_error)) {
+                            !mbar_wait(smem_u32(kv_empty + slot2), (L / C::kSlots - 1) & 1, a.dev_error)) {
                             ok = false;
                             break;
                         }
-                        const uint32_t fb = smem_u32(kv_full + slot);
-                        mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * kRowBytes * C::kHalves));
-                        const uint32_t dst = ring + slot * C::kTileBytes;
+                        const uint32_t fb = smem_u32(kv_full + slot2);
+                        if (lane == 0) mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * kRowBytes * C::kHalves));
+                        const uint32_t dst = ring + slot2 * C::kTileBytes;
                         for (int b = 0; b < nbox; ++b) {
                             const int tok = key0 + b * box;
-                            const int blk = __ldg(bt + tok / B);
-                            int row;
-                            if ((unsigned)blk < (unsigned)a.num_blocks) {
-                                row = blk * B + (tok % B);
-                            } else {
-                                report(a.dev_error, PA_DEVERR_BLOCK_ID);
-                                row = -box;     // fully out of range: TMA fills zeros
-                            }
+                            const int blk = __shfl_sync(0xffffffffu, ids, tok / B - chunk);
+                            if (lane == 0) {
+                                int row;
+                                if ((unsigned)blk < (unsigned)a.num_blocks) {
+                                    row = blk * B + (tok % B);
+                                } else {
+                                    report(a.dev_error, PA_DEVERR_BLOCK_ID);
+                                    row = -box;     // fully out of range: TMA fills zeros
+                                }
 #pragma unroll
-                            for (int h = 0; h < C::kHalves; ++h)
-                                tma_load_3d(dst + h * kSlab + b * box * kRowBytes, kv ? &tm_v : &tm_k, h * 64, U.kvh,
-                                            row, fb);
+                                for (int h = 0; h < C::kHalves; ++h)
+                                    tma_load_3d(dst + h * kSlab + b * box * kRowBytes, kv ? &tm_v : &tm_k, h * 64,
+                                                U.kvh, row, fb);
+                            }
                         }
                     }
                 }
             }
+            next = decode(next_u);
         }
+        // Leave no TMA copy in flight: wait (bounded) for the last load of every ring slot and for the
+        // last Q load.  On the normal path the MMA warp consumed them all and these return at once.
+        for (uint32_t i = (L > (uint32_t)C::kSlots ? L - C::kSlots : 0); i < L; ++i)
+            mbar_wait(smem_u32(kv_full + i % C::kSlots), (i / C::kSlots) & 1, a.dev_error);
+        if (nq > 0) mbar_wait(smem_u32(q_full), (nq - 1) & 1, a.dev_error);
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA ==
         constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kN, 0, 0);
@@ -387,15 +433,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto wait_slot = [&](uint32_t idx) -> bool {
             return mbar_wait(smem_u32(kv_full + idx % C::kSlots), (idx / C::kSlots) & 1, a.dev_error);
         };
+        // Descriptors are built once; an MMA only adds a byte offset (>> 4) to the start-address field
+        // (14 bits of a 256 KB window, so the add never carries into the other fields).
+        const uint64_t q_desc = smem_desc_sw128(q_s, 16, 1024);
+        const uint64_t k_desc = smem_desc_sw128(ring, 16, 1024);
+        const uint64_t v_desc = smem_desc_sw128(ring, kSlab, 1024);
         auto issue_s = [&](int x, uint32_t kidx) {
             if (lane == 0) {
-                const uint32_t ks = ring + (kidx % C::kSlots) * C::kTileBytes;
-                const uint32_t qs = q_s + x * C::kTileBytes;
+                const uint64_t qd = q_desc + ((uint32_t)(x * C::kTileBytes) >> 4);
+                const uint64_t kd = k_desc + (((kidx % C::kSlots) * (uint32_t)C::kTileBytes) >> 4);
+                const uint32_t d = tmem + col_s(x);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(qs + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(ks + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
-                    tc_mma_ss(tmem + col_s(x), ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk >> 2) * kSlab + (kk & 3) * 32) >> 4;
+                    tc_mma_ss(d, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(smem_u32(s_full + x));
             }
@@ -403,13 +454,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         auto issue_pv = [&](int x, uint32_t vidx, bool accumulate) {
             if (lane == 0) {
-                const uint32_t vs = ring + (vidx % C::kSlots) * C::kTileBytes;
-                const uint32_t ps = p_s + x * C::kPBytes;
+                const uint64_t vd = v_desc + (((vidx % C::kSlots) * (uint32_t)C::kTileBytes) >> 4);
+                const uint32_t d = tmem + col_o(x), pa = tmem + col_s(x);
 #pragma unroll
                 for (int kk = 0; kk < kN / 16; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(ps + (kk >> 2) * kSlab + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(vs + kk * 16 * kRowBytes, kSlab, 1024);
-                    tc_mma_ss(tmem + col_o(x), ad, bd, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+                    // A = P_X in TMEM: 16 keys = 8 columns of packed bf16 pairs; B = V rows kk*16 ..
+                    tc_mma_ts(d, pa + kk * 8, vd + ((kk * 16 * kRowBytes) >> 4), idesc_pv,
+                              (accumulate || kk > 0) ? 1u : 0u);
                 }
             }
             __syncwarp();
@@ -532,24 +583,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     rescale = true;
                 }
                 const float neg = -m_ref;
-                // P = exp2(s * scale_log2 - m_ref) as bf16, stored 8 keys (16 bytes) at a time
+                // P = exp2(s * scale_log2 - m_ref) as packed bf16 pairs, written over the S_X columns already
+                // read (32 keys = 16 columns per store)
                 float ls[4] = {0.f, 0.f, 0.f, 0.f};
-                const uint32_t pb = p_s + x * C::kPBytes;
 #pragma unroll
-                for (int kc = 0; kc < kN / 8; ++kc) {
-                    uint32_t w[4];
+                for (int kc = 0; kc < kN / 32; ++kc) {
+                    uint32_t w[16];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int e = kc * 8 + 2 * i;
+                    for (int i = 0; i < 16; ++i) {
+                        const int e = kc * 32 + 2 * i;
                         const float p0 = fast_exp2(fmaf(__uint_as_float(sr[e >> 5][e & 31]), sl, neg));
                         const float p1 = fast_exp2(fmaf(__uint_as_float(sr[e >> 5][(e + 1) & 31]), sl, neg));
                         w[i] = pack_bf16(p0, p1);
-                        ls[i] += p0 + p1;
+                        ls[i & 3] += p0 + p1;
                     }
-                    const uint32_t dst = pb + (kc >> 3) * kSlab + swz128(r, kc & 7);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w[0]), "r"(w[1]),
-                                 "r"(w[2]), "r"(w[3])
-                                 : "memory");
+                    tmem_st16(lane_base + col_s(x) + kc * 16, w);
                 }
                 l = l * corr + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
                 if (rescale && j > 0) {
@@ -565,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_wait_st();
                 }
-                fence_proxy_async_smem();
+                tc_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(p_full + x));
@@ -655,10 +703,11 @@ cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &tm_q, cons
 
 }  // namespace
 
-size_t prefill_workspace_bytes(int32_t batch, int32_t max_seqlen_q, int32_t group) {
+size_t prefill_workspace_bytes(int32_t batch, int32_t max_seqlen_q, int32_t group, int32_t num_kv_heads) {
     const int32_t TQ = kM / group;
     const int64_t R = ((int64_t)max_seqlen_q + 2 * TQ - 1) / (2 * TQ);
-    const size_t words = 16 + (size_t)(R + 1) + (size_t)batch;
+    const PlanLayout lay = plan_layout((int32_t)R, batch);
+    const size_t words = (size_t)lay.units + (size_t)4 * R * batch * num_kv_heads;
     return (words * sizeof(int32_t) + 255) / 256 * 256;
 }
 

@@ -47,7 +47,8 @@ constexpr int kM = 128;                // MMA rows per Q tile
 constexpr int kN = 128;                // keys per K/V tile
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;          // 2 softmax warpgroups + TMA warp + MMA warp
+constexpr int kFixWarp = 10;
+constexpr int kThreads = 352;          // 2 softmax warpgroups + TMA warp + MMA warp + V-fix warp
 constexpr int kRowBytes = 128;         // one 64-element bf16 swizzle row
 constexpr int kSlab = kM * kRowBytes;  // 128 rows x 128 B = 16 KB
 constexpr int kUnitQueue = 4;          // unit ids handed from the TMA warp to the other roles
@@ -62,7 +63,8 @@ struct PrefillCfg {
     static constexpr int kRingOff = kQOff + 2 * kTileBytes;
     static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
     // kv_full[S] kv_empty[S] q_full q_empty s_full[2] p_full[2] o_full[2] o_empty[2] done uq_full[4] uq_empty[4]
-    static constexpr int kNumBars = 2 * kSlots + 11 + 2 * kUnitQueue;
+    // v_fixed vlast_full[2]
+    static constexpr int kNumBars = 2 * kSlots + 11 + 2 * kUnitQueue + 3;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 64 + kUnitQueue * 64 + 1024;
     static constexpr uint32_t kTmemCols = 512;                  // S_A 0, O_A 128, S_B 256, O_B 384
                                                                 // (P_X, bf16, overwrites the first 64 columns of S_X)
@@ -260,6 +262,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *done = o_empty + 2;
     uint64_t *uq_full = done + 1;      // [kUnitQueue]
     uint64_t *uq_empty = uq_full + kUnitQueue;
+    uint64_t *v_fixed = uq_empty + kUnitQueue;   // the last V tile of a unit is ready for PV
+    // The last V tile of a unit lands on its own barrier, alternating by unit: the TMA warp runs at most
+    // one unit ahead of the V-fix warp (the next unit's loads wait for this unit's S products, and those
+    // wait for the fix), so two barriers keep every phase distinct.
+    uint64_t *vlast_full = v_fixed + 1;           // [2]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
     // unit queue: kUnitQueue entries of 16 words (a decoded Unit; valid = -1 ends the stream)
     volatile int32_t *unit_q = reinterpret_cast<volatile int32_t *>(tmem_slot + 16);
@@ -288,9 +295,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(o_empty + x), 4);
         }
         mbar_init(smem_u32(done), 1);
+        mbar_init(smem_u32(v_fixed), 1);
+        mbar_init(smem_u32(vlast_full), 1);
+        mbar_init(smem_u32(vlast_full + 1), 1);
         for (int i = 0; i < kUnitQueue; ++i) {
             mbar_init(smem_u32(uq_full + i), 1);
-            mbar_init(smem_u32(uq_empty + i), 9);   // the MMA warp and the eight softmax warps
+            mbar_init(smem_u32(uq_empty + i), 10);  // the MMA warp, the V-fix warp, the eight softmax warps
         }
         fence_barrier_init();
     }
@@ -345,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int4 rec = units[u];
             return unit_from_record(a, rec, geo[rec.x], TQ);
         };
-        uint32_t nq = 0, L = 0;
+        uint32_t nq = 0, L = 0, nvlast = 0;
         bool ok = true;
         Unit next = decode(fetch());
         for (uint32_t nu = 0;; ++nu) {
@@ -379,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int32_t *bt = a.block_table + (int64_t)U.s * a.bt_stride;
                 const int kend = max(U.kend[0], U.kend[1]);
                 int chunk = -32, ids = 0;            // block_table[chunk + lane] lives in `ids` of that lane
+                if (ok && U.nk > 0) ++nvlast;
                 for (int j = 0; j < U.nk && ok; ++j) {
                     const int key0 = j * kN;
                     const int nbox = (min(kN, kend - key0) + box - 1) / box;
@@ -394,8 +405,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ok = false;
                             break;
                         }
-                        const uint32_t fb = smem_u32(kv_full + slot2);
-                        if (lane == 0) mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * kRowBytes * C::kHalves));
+                        // the last V tile of the unit lands on its own barrier (the V-fix warp consumes it in
+                        // order); the ring slot's barrier still completes one phase, with no bytes
+                        const bool vlast = kv == 1 && j == U.nk - 1;
+                        const uint32_t fb = smem_u32(vlast ? vlast_full + ((nvlast - 1) & 1) : kv_full + slot2);
+                        if (lane == 0) {
+                            if (vlast) mbar_arrive(smem_u32(kv_full + slot2));
+                            mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * kRowBytes * C::kHalves));
+                        }
                         const uint32_t dst = ring + slot2 * C::kTileBytes;
                         for (int b = 0; b < nbox; ++b) {
                             const int tok = key0 + b * box;
@@ -424,22 +441,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (uint32_t i = (L > (uint32_t)C::kSlots ? L - C::kSlots : 0); i < L; ++i)
             mbar_wait(smem_u32(kv_full + i % C::kSlots), (i / C::kSlots) & 1, a.dev_error);
         if (nq > 0) mbar_wait(smem_u32(q_full), (nq - 1) & 1, a.dev_error);
+        for (uint32_t i = (nvlast > 2 ? nvlast - 2 : 0); i < nvlast; ++i)
+            mbar_wait(smem_u32(vlast_full + (i & 1)), (i >> 1) & 1, a.dev_error);
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA ==
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kN, 0, 0);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, D, 0, 1);
-        uint32_t nq = 0, L = 0, np[2] = {0, 0}, no[2] = {0, 0};
-        bool ok = true;
-        auto wait_slot = [&](uint32_t idx) -> bool {
-            return mbar_wait(smem_u32(kv_full + idx % C::kSlots), (idx / C::kSlots) & 1, a.dev_error);
-        };
-        // Descriptors are built once; an MMA only adds a byte offset (>> 4) to the start-address field
-        // (14 bits of a 256 KB window, so the add never carries into the other fields).
-        const uint64_t q_desc = smem_desc_sw128(q_s, 16, 1024);
-        const uint64_t k_desc = smem_desc_sw128(ring, 16, 1024);
-        const uint64_t v_desc = smem_desc_sw128(ring, kSlab, 1024);
-        auto issue_s = [&](int x, uint32_t kidx) {
-            if (lane == 0) {
+        // One thread: the tensor cores keep almost no queue, so this thread does nothing but wait for
+        // its operands and issue.  Order per key tile j: PV_A(j) S_A(j+1) PV_B(j) S_B(j+1).
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kN, 0, 0);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, D, 0, 1);
+            uint32_t nq = 0, L = 0, np[2] = {0, 0}, no[2] = {0, 0}, nfix = 0;
+            bool ok = true;
+            // Descriptors are built once; an MMA only adds a byte offset (>> 4) to the start-address
+            // field (14 bits of a 256 KB window, so the add never carries into the other fields).
+            const uint64_t q_desc = smem_desc_sw128(q_s, 16, 1024);
+            const uint64_t k_desc = smem_desc_sw128(ring, 16, 1024);
+            const uint64_t v_desc = smem_desc_sw128(ring, kSlab, 1024);
+            auto wait_slot = [&](uint32_t idx) -> bool {
+                return mbar_wait(smem_u32(kv_full + idx % C::kSlots), (idx / C::kSlots) & 1, a.dev_error);
+            };
+            auto issue_s = [&](int x, uint32_t kidx) {
                 const uint64_t qd = q_desc + ((uint32_t)(x * C::kTileBytes) >> 4);
                 const uint64_t kd = k_desc + (((kidx % C::kSlots) * (uint32_t)C::kTileBytes) >> 4);
                 const uint32_t d = tmem + col_s(x);
@@ -449,11 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_mma_ss(d, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(smem_u32(s_full + x));
-            }
-            __syncwarp();
-        };
-        auto issue_pv = [&](int x, uint32_t vidx, bool accumulate) {
-            if (lane == 0) {
+            };
+            auto issue_pv = [&](int x, uint32_t vidx, bool accumulate) {
                 const uint64_t vd = v_desc + (((vidx % C::kSlots) * (uint32_t)C::kTileBytes) >> 4);
                 const uint32_t d = tmem + col_o(x), pa = tmem + col_s(x);
 #pragma unroll
@@ -462,81 +480,103 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_mma_ts(d, pa + kk * 8, vd + ((kk * 16 * kRowBytes) >> 4), idesc_pv,
                               (accumulate || kk > 0) ? 1u : 0u);
                 }
-            }
-            __syncwarp();
-        };
-        auto commit = [&](uint64_t *bar) {
-            if (lane == 0) tc_commit(smem_u32(bar));
-            __syncwarp();
-        };
-        for (uint32_t k = 0; ok; ++k) {
-            Unit U;
-            if (!pop_unit(k, lane == 0, U)) break;
-            if (!U.valid) continue;
-            if (!mbar_wait(smem_u32(q_full), nq & 1, a.dev_error)) break;
-            ++nq;
-            const bool hasB = U.nt[1] > 0;
-            // K_0: S_A(0), S_B(0)
-            if (!wait_slot(L)) break;
-            tc_fence_after();
-            issue_s(0, L);
-            if (hasB) issue_s(1, L);
-            commit(kv_empty + L % C::kSlots);
-            if (U.nk == 1) commit(q_empty);
-            for (int j = 0; j < U.nk && ok; ++j) {
-                const uint32_t vidx = L + 2 * j + 1, knext = L + 2 * j + 2;
-                if (!wait_slot(vidx)) { ok = false; break; }
-                if (j == U.nk - 1) {
-                    // zero V rows past the unit's key range (stale or poisoned slots)
-                    const int valid = max(U.kend[0], U.kend[1]) - j * kN;
-                    if (valid < kN) {
-                        const uint32_t vs = ring + (vidx % C::kSlots) * C::kTileBytes;
-                        for (int e = lane; e < (kN - valid) * C::kHalves * 8; e += 32) {
-                            const int r = valid + e / (C::kHalves * 8);
-                            const int h = (e / 8) % C::kHalves, ch = e % 8;
-                            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(
-                                             vs + h * kSlab + r * kRowBytes + ch * 16),
-                                         "r"(0u)
-                                         : "memory");
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                    }
+            };
+            for (uint32_t k = 0; ok; ++k) {
+                const int slot = k % kUnitQueue;
+                if (!mbar_wait(smem_u32(uq_full + slot), (k / kUnitQueue) & 1, a.dev_error)) break;
+                Unit U;
+                {
+                    int32_t *dst = reinterpret_cast<int32_t *>(&U);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) dst[i] = unit_q[slot * 16 + i];
                 }
-                bool knext_ready = false;
-                for (int x = 0; x < 2; ++x) {
-                    if (j >= U.nt[x]) continue;
-                    if (!mbar_wait(smem_u32(p_full + x), np[x] & 1, a.dev_error)) { ok = false; break; }
-                    ++np[x];
-                    if (j == 0 && no[x] > 0 && !mbar_wait(smem_u32(o_empty + x), (no[x] - 1) & 1, a.dev_error)) {
+                mbar_arrive(smem_u32(uq_empty + slot));
+                if (U.valid < 0) break;
+                if (!U.valid) continue;
+                if (!mbar_wait(smem_u32(q_full), nq & 1, a.dev_error)) break;
+                ++nq;
+                const bool hasB = U.nt[1] > 0;
+                // K_0: S_A(0), S_B(0)
+                if (!wait_slot(L)) break;
+                tc_fence_after();
+                issue_s(0, L);
+                if (hasB) issue_s(1, L);
+                tc_commit(smem_u32(kv_empty + L % C::kSlots));
+                if (U.nk == 1) tc_commit(smem_u32(q_empty));
+                for (int j = 0; j < U.nk && ok; ++j) {
+                    const uint32_t vidx = L + 2 * j + 1, knext = L + 2 * j + 2;
+                    if (j == U.nk - 1) {
+                        // the V-fix warp has zeroed the rows past the key range of the unit's last V tile
+                        if (!mbar_wait(smem_u32(v_fixed), nfix & 1, a.dev_error)) { ok = false; break; }
+                        ++nfix;
+                    } else if (!wait_slot(vidx)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    issue_pv(x, vidx, j > 0);
-                    if (j == U.nt[x] - 1) {
-                        commit(o_full + x);
-                        ++no[x];
-                    }
-                    if (j + 1 < U.nt[x]) {
-                        if (!knext_ready) {
-                            if (!wait_slot(knext)) { ok = false; break; }
-                            tc_fence_after();
-                            knext_ready = true;
+                    bool knext_ready = false;
+                    for (int x = 0; x < 2; ++x) {
+                        if (j >= U.nt[x]) continue;
+                        if (!mbar_wait(smem_u32(p_full + x), np[x] & 1, a.dev_error)) { ok = false; break; }
+                        ++np[x];
+                        if (j == 0 && no[x] > 0 &&
+                            !mbar_wait(smem_u32(o_empty + x), (no[x] - 1) & 1, a.dev_error)) {
+                            ok = false;
+                            break;
                         }
-                        issue_s(x, knext);
+                        tc_fence_after();
+                        issue_pv(x, vidx, j > 0);
+                        if (j == U.nt[x] - 1) {
+                            tc_commit(smem_u32(o_full + x));
+                            ++no[x];
+                        }
+                        if (j + 1 < U.nt[x]) {
+                            if (!knext_ready) {
+                                if (!wait_slot(knext)) { ok = false; break; }
+                                tc_fence_after();
+                                knext_ready = true;
+                            }
+                            issue_s(x, knext);
+                        }
                     }
+                    if (!ok) break;
+                    tc_commit(smem_u32(kv_empty + vidx % C::kSlots));
+                    if (knext_ready) tc_commit(smem_u32(kv_empty + knext % C::kSlots));
+                    if (j == U.nk - 2) tc_commit(smem_u32(q_empty));   // every S product of the unit is issued
                 }
-                if (!ok) break;
-                commit(kv_empty + vidx % C::kSlots);
-                if (knext_ready) commit(kv_empty + knext % C::kSlots);
-                if (j == U.nk - 2) commit(q_empty);   // every S product of the unit is issued
+                L += 2 * U.nk;
             }
-            L += 2 * U.nk;
+            // every MMA issued by this thread has completed before TMEM is freed
+            tc_commit(smem_u32(done));
+            mbar_wait(smem_u32(done), 0, a.dev_error);
         }
-        // every MMA issued by this thread has completed before TMEM is freed
-        commit(done);
-        mbar_wait(smem_u32(done), 0, a.dev_error);
+    } else if (warp == kFixWarp) {
+        // ========================================================== V fix ==
+        // Zero the rows of each unit's last V tile past its key range (stale or poisoned cache slots),
+        // so that masked keys, whose probabilities are exactly 0, never meet a NaN.
+        uint32_t L = 0, nfx = 0;
+        for (uint32_t k = 0;; ++k) {
+            Unit U;
+            if (!pop_unit(k, lane == 0, U)) break;
+            if (!U.valid) continue;
+            const uint32_t vidx = L + 2 * (U.nk - 1) + 1;
+            L += 2 * U.nk;
+            if (!mbar_wait(smem_u32(vlast_full + (nfx & 1)), (nfx >> 1) & 1, a.dev_error)) break;
+            ++nfx;
+            const int valid = max(U.kend[0], U.kend[1]) - (U.nk - 1) * kN;
+            if (valid < kN) {
+                const uint32_t vs = ring + (vidx % C::kSlots) * C::kTileBytes;
+                for (int e = lane; e < (kN - valid) * C::kHalves * 8; e += 32) {
+                    const int r = valid + e / (C::kHalves * 8);
+                    const int h = (e / 8) % C::kHalves, ch = e % 8;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(vs + h * kSlab + r * kRowBytes + ch * 16),
+                                 "r"(0u)
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(v_fixed));
+        }
     } else {
         // ======================================================== softmax ==
         const int x = warp >> 2;                       // 0: tile A, 1: tile B

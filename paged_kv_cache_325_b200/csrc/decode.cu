@@ -48,13 +48,45 @@ struct DecodeCfg {
     static constexpr int kKvBytes = kHalves * kHalfBytes;        // K (or V) part of a stage
     static constexpr int kStageBytes = 2 * kKvBytes;
     static constexpr int kRingBytes = kStages * kStageBytes;
-    static constexpr int kRedBytes = kConsumerWarps * 16 * (D + 2) * 4;
-    static_assert(kRedBytes <= kRingBytes, "reduction scratch must fit in the ring");
-    static constexpr int kSmemBytes = kRingBytes + 2 * kStages * 8 + 1024;  // + barriers + alignment slack
+    static constexpr int kBarOff = kRingBytes;                   // 256 bytes of barriers
+    static constexpr int kQOff = kBarOff + 256;                  // 2 slots of the group's G q-head rows
+    // then the merge area: per consumer warp, G rows of D partial sums plus (max, sum)
+    static constexpr size_t red_off(int G) { return (size_t)kQOff + 2 * (size_t)G * D * 2; }
+    static constexpr size_t smem_bytes(int G) {
+        return red_off(G) + (size_t)kConsumerWarps * G * (D + 2) * 4 + 1024;
+    }
 };
 
 __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+
+// A work item is (split, sequence, KV head); items are numbered split-major and dealt round-robin to
+// persistent CTAs, so every CTA streams several items through one continuous TMA ring.
+struct DecItem {
+    int valid;          // 0: skip (past the context, or an invalid context length)
+    int s, kvh, t_begin, t_end, ntiles, split;
+};
+
+__device__ __forceinline__ DecItem dec_item(const DecodeArgs &a, int i, bool report_bad) {
+    DecItem it;
+    const int per_split = a.batch * a.num_kv_heads;
+    it.split = i / per_split;
+    const int r = i % per_split;
+    it.s = r / a.num_kv_heads;
+    it.kvh = r % a.num_kv_heads;
+    it.valid = 0;
+    const int ctx = __ldg(a.context_lens + it.s);
+    if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size) {
+        if (report_bad && it.split == 0 && it.kvh == 0) report(a.dev_error, PA_DEVERR_CONTEXT_LEN);
+        return it;
+    }
+    it.t_begin = it.split * a.plan.chunk;
+    if (it.t_begin >= ctx) return it;            // this split lies past the end of the context
+    it.t_end = min(ctx, it.t_begin + a.plan.chunk);
+    it.ntiles = (it.t_end - it.t_begin + kTile - 1) / kTile;
+    it.valid = 1;
+    return it;
 }
 
 template <int D>
@@ -64,250 +96,283 @@ __global__ void __launch_bounds__(kThreads, 2)
     using C = DecodeCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kRingBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *empty = full + C::kStages;
+    uint64_t *qfull = empty + C::kStages;       // [2]
+    uint64_t *qempty = qfull + 2;               // [2]
+    const int G = a.group;
+    float *red_o = reinterpret_cast<float *>(smem + C::red_off(G));   // [warp][G][D]
+    float *red_ml = red_o + kConsumerWarps * G * D;                 // [warp][G][2]
 
-    const int split = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ctx = __ldg(a.context_lens + s);
-    if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size) {
-        if (split == 0 && kvh == 0 && threadIdx.x == 0) report(a.dev_error, PA_DEVERR_CONTEXT_LEN);
-        return;
-    }
-    const int t_begin = split * a.plan.chunk;
-    if (t_begin >= ctx) return;               // this split lies past the end of the context
-    const int t_end = min(ctx, t_begin + a.plan.chunk);
-    const int ntiles = (t_end - t_begin + kTile - 1) / kTile;
+    const int n_items = a.plan.max_splits * a.batch * a.num_kv_heads;
+    const uint32_t ring = smem_u32(smem);
+    const uint32_t qsm = ring + C::kQOff;
+    const uint32_t qslot = (uint32_t)(G * D * 2);
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < C::kStages; ++st) {
             mbar_init(smem_u32(full + st), 1);
             mbar_init(smem_u32(empty + st), kConsumerWarps);
         }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(qfull + i), 1);
+            mbar_init(smem_u32(qempty + i), kConsumerWarps);
+        }
         fence_barrier_init();
     }
     __syncthreads();
-
-    const uint32_t ring = smem_u32(smem);
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------ producer --
         if (lane == 0) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            const int32_t *bt = a.block_table + (int64_t)s * a.bt_stride;
             const int B = a.block_size, box = a.box_tokens;
-            int issued = 0;
-            for (int i = 0; i < ntiles; ++i) {
-                const int st = i % C::kStages;
-                if (i >= C::kStages && !mbar_wait(smem_u32(empty + st), ((i / C::kStages) & 1) ^ 1, a.dev_error))
-                    break;
-                const int tile0 = t_begin + i * kTile;
-                const int nbox = (min(kTile, t_end - tile0) + box - 1) / box;
-                const uint32_t fb = smem_u32(full + st);
-                mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * 128 * C::kHalves * 2));
-                const uint32_t kdst = ring + st * C::kStageBytes;
-                const uint32_t vdst = kdst + C::kKvBytes;
-                for (int b = 0; b < nbox; ++b) {
-                    const int tok = tile0 + b * box;
-                    const int blk = __ldg(bt + tok / B);
-                    int row;
-                    if ((unsigned)blk < (unsigned)a.num_blocks) {
-                        row = blk * B + (tok % B);
-                    } else {               // out-of-range id: load zeros instead (TMA fills)
-                        report(a.dev_error, PA_DEVERR_BLOCK_ID);
-                        row = -box;
+            uint32_t gt = 0, nqi = 0;             // tiles and Q copies issued so far
+            bool ok = true;
+            for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x) {
+                const DecItem it = dec_item(a, i, true);
+                if (!it.valid) continue;
+                // Q rows of the GQA group: one contiguous bulk copy
+                const int qs = nqi & 1;
+                if (nqi >= 2 && !mbar_wait(smem_u32(qempty + qs), ((nqi >> 1) - 1) & 1, a.dev_error)) break;
+                const uint32_t qbytes = (uint32_t)(G * D * 2);
+                mbar_arrive_expect_tx(smem_u32(qfull + qs), qbytes);
+                bulk_load(qsm + qs * qslot,
+                          static_cast<const __nv_bfloat16 *>(a.q) + ((int64_t)it.s * a.num_q_heads + (int64_t)it.kvh * G) * D,
+                          qbytes, smem_u32(qfull + qs));
+                ++nqi;
+                const int32_t *bt = a.block_table + (int64_t)it.s * a.bt_stride;
+                for (int t = 0; t < it.ntiles; ++t, ++gt) {
+                    const int st = gt % C::kStages;
+                    if (gt >= (uint32_t)C::kStages &&
+                        !mbar_wait(smem_u32(empty + st), ((gt / C::kStages) & 1) ^ 1, a.dev_error)) {
+                        ok = false;
+                        break;
                     }
+                    const int tile0 = it.t_begin + t * kTile;
+                    const int nbox = (min(kTile, it.t_end - tile0) + box - 1) / box;
+                    const uint32_t fb = smem_u32(full + st);
+                    mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * 128 * C::kHalves * 2));
+                    const uint32_t kdst = ring + st * C::kStageBytes;
+                    const uint32_t vdst = kdst + C::kKvBytes;
+                    for (int b = 0; b < nbox; ++b) {
+                        const int tok = tile0 + b * box;
+                        const int blk = __ldg(bt + tok / B);
+                        int row;
+                        if ((unsigned)blk < (unsigned)a.num_blocks) {
+                            row = blk * B + (tok % B);
+                        } else {               // out-of-range id: load zeros instead (TMA fills)
+                            report(a.dev_error, PA_DEVERR_BLOCK_ID);
+                            row = -box;
+                        }
 #pragma unroll
-                    for (int h = 0; h < C::kHalves; ++h) {
-                        const uint32_t off = h * kHalfBytes + b * box * 128;
-                        tma_load_3d(kdst + off, &tm_k, h * 64, kvh, row, fb);
-                        tma_load_3d(vdst + off, &tm_v, h * 64, kvh, row, fb);
+                        for (int h = 0; h < C::kHalves; ++h) {
+                            const uint32_t off = h * kHalfBytes + b * box * 128;
+                            tma_load_3d(kdst + off, &tm_k, h * 64, it.kvh, row, fb);
+                            tma_load_3d(vdst + off, &tm_v, h * 64, it.kvh, row, fb);
+                        }
                     }
                 }
-                issued = i + 1;
             }
-            // leave no TMA copy in flight: wait (bounded) for the last load of every stage; on the normal path
-            // the consumers have already waited for them all and these return at once
-            for (int i = (issued > C::kStages ? issued - C::kStages : 0); i < issued; ++i)
+            // leave no copy in flight: wait (bounded) for the last load of every stage and the last Q copies;
+            // on the normal path the consumers have already waited for them all and these return at once
+            for (uint32_t i = (gt > (uint32_t)C::kStages ? gt - C::kStages : 0); i < gt; ++i)
                 mbar_wait(smem_u32(full + i % C::kStages), (i / C::kStages) & 1, a.dev_error);
+            for (uint32_t i = (nqi > 2 ? nqi - 2 : 0); i < nqi; ++i)
+                mbar_wait(smem_u32(qfull + (i & 1)), (i >> 1) & 1, a.dev_error);
         }
         return;
     }
 
     // ---------------------------------------------------------- consumers --
-    const int G = a.group;
     const int g0 = lane >> 2;             // accumulator rows g0 and g0 + 8
     const int c2 = (lane & 3) * 2;        // accumulator columns c2, c2 + 1
-    uint32_t qa[D / 16][4];
-    {
-        const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(a.q) +
-                                  ((int64_t)s * a.num_q_heads + (int64_t)kvh * G) * D;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            const int k0 = ks * 16 + c2;
-            qa[ks][0] = g0 < G ? __ldg(reinterpret_cast<const uint32_t *>(qb + g0 * D + k0)) : 0u;
-            qa[ks][1] = g0 + 8 < G ? __ldg(reinterpret_cast<const uint32_t *>(qb + (g0 + 8) * D + k0)) : 0u;
-            qa[ks][2] = g0 < G ? __ldg(reinterpret_cast<const uint32_t *>(qb + g0 * D + k0 + 8)) : 0u;
-            qa[ks][3] = g0 + 8 < G ? __ldg(reinterpret_cast<const uint32_t *>(qb + (g0 + 8) * D + k0 + 8)) : 0u;
-        }
-    }
-
-    float m_run[2] = {-INFINITY, -INFINITY};
-    float l_run[2] = {0.f, 0.f};
-    float o[D / 8][4];
-#pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-
     const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: matrix index / row this lane addresses
+    const bool single = a.plan.max_splits == 1;
+    uint32_t gt = 0, nqi = 0;
     bool ok = true;
-    for (int i = 0; i < ntiles; ++i) {
-        const int st = i % C::kStages;
-        const bool landed = mbar_wait(smem_u32(full + st), (i / C::kStages) & 1, a.dev_error);
-        if (!__all_sync(0xffffffffu, landed)) {   // leave together: the loop body uses full-warp shuffles
-            ok = false;
-            break;
+    for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
+        const DecItem it = dec_item(a, i, false);
+        if (!it.valid) continue;
+        // Q fragments; rows past the group are zero
+        const int qs = nqi & 1;
+        // After a timed-out wait the consumers keep the same control flow (every warp must still reach
+        // the merge barriers) but stop waiting; the results are garbage and dev_error says so.
+        {
+            const bool landed = ok && mbar_wait(smem_u32(qfull + qs), (nqi >> 1) & 1, a.dev_error);
+            if (!__all_sync(0xffffffffu, landed)) ok = false;
         }
-        const uint32_t kbase = ring + st * C::kStageBytes;
-        const uint32_t vbase = kbase + C::kKvBytes;
-        const int tok0 = t_begin + i * kTile + warp * 16;   // first token of this warp's slice
-
-        // S = Q K^T over this warp's 16 tokens (two n-tiles of 8 tokens)
-        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        ++nqi;
+        uint32_t qa[D / 16][4];
+        {
+            const uint32_t qb = qsm + qs * qslot;
+            const bool r0 = g0 < G, r1 = g0 + 8 < G;
+            const uint32_t a0 = qb + (r0 ? g0 : 0) * D * 2, a1 = qb + (r1 ? g0 + 8 : 0) * D * 2;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            const int trow = warp * 16 + (mi >> 1) * 8 + mr;
-            const int dch = ks * 2 + (mi & 1);
-            uint32_t b0n0, b1n0, b0n1, b1n1;
-            ldmatrix_x4(kbase + (dch >> 3) * kHalfBytes + swz128(trow, dch & 7), b0n0, b1n0, b0n1, b1n1);
-            mma_bf16_16816(sc[0], qa[ks], b0n0, b1n0);
-            mma_bf16_16816(sc[1], qa[ks], b0n1, b1n1);
-        }
-
-        // scale into log2 units and select out positions past the end
-        const bool partial = tok0 + 16 > t_end;
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int tok = tok0 + n * 8 + c2 + (e & 1);
-                const float v = sc[n][e] * a.scale_log2;
-                sc[n][e] = (!partial || tok < t_end) ? v : -INFINITY;
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t k0 = (ks * 16 + c2) * 2;
+                uint32_t v0, v1, v2, v3;
+                asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v0) : "r"(a0 + k0));
+                asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v1) : "r"(a1 + k0));
+                asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v2) : "r"(a0 + k0 + 16));
+                asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v3) : "r"(a1 + k0 + 16));
+                qa[ks][0] = r0 ? v0 : 0u;
+                qa[ks][1] = r1 ? v1 : 0u;
+                qa[ks][2] = r0 ? v2 : 0u;
+                qa[ks][3] = r1 ? v3 : 0u;
             }
-
-        // online softmax (rows g0 and g0 + 8)
-        float mx[2];
-        mx[0] = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-        mx[1] = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-        }
-        float corr[2], ref[2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const float m_new = fmaxf(m_run[r], mx[r]);
-            ref[r] = m_new == -INFINITY ? 0.f : m_new;
-            corr[r] = fast_exp2(m_run[r] - ref[r]);
-            m_run[r] = m_new;
-        }
-        float p[2][4];
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) p[n][e] = fast_exp2(sc[n][e] - ref[e >> 1]);
-        l_run[0] = l_run[0] * corr[0] + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
-        l_run[1] = l_run[1] * corr[1] + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
-        if (!__all_sync(0xffffffffu, corr[0] == 1.f && corr[1] == 1.f)) {
-#pragma unroll
-            for (int nt = 0; nt < D / 8; ++nt) {
-                o[nt][0] *= corr[0];
-                o[nt][1] *= corr[0];
-                o[nt][2] *= corr[1];
-                o[nt][3] *= corr[1];
-            }
-        }
-        uint32_t pa[4];
-        pa[0] = pack_bf16(p[0][0], p[0][1]);
-        pa[1] = pack_bf16(p[0][2], p[0][3]);
-        pa[2] = pack_bf16(p[1][0], p[1][1]);
-        pa[3] = pack_bf16(p[1][2], p[1][3]);
-
-        // V fragments hold tokens tok0 + c2 + {0,1} (b0) and tok0 + 8 + c2 + {0,1} (b1)
-        uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
-        if (partial) {
-            vm0 = (tok0 + c2 < t_end ? 0x0000ffffu : 0u) | (tok0 + c2 + 1 < t_end ? 0xffff0000u : 0u);
-            vm1 = (tok0 + 8 + c2 < t_end ? 0x0000ffffu : 0u) | (tok0 + 9 + c2 < t_end ? 0xffff0000u : 0u);
-        }
-#pragma unroll
-        for (int jp = 0; jp < D / 16; ++jp) {
-            const int trow = warp * 16 + (mi & 1) * 8 + mr;
-            const int dch = jp * 2 + (mi >> 1);
-            uint32_t b0a, b1a, b0b, b1b;
-            ldmatrix_x4_trans(vbase + (dch >> 3) * kHalfBytes + swz128(trow, dch & 7), b0a, b1a, b0b, b1b);
-            b0a &= vm0;
-            b1a &= vm1;
-            b0b &= vm0;
-            b1b &= vm1;
-            mma_bf16_16816(o[2 * jp], pa, b0a, b1a);
-            mma_bf16_16816(o[2 * jp + 1], pa, b0b, b1b);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(empty + st));
-    }
+        if (lane == 0) mbar_arrive(smem_u32(qempty + qs));
 
+        float m_run[2] = {-INFINITY, -INFINITY};
+        float l_run[2] = {0.f, 0.f};
+        float o[D / 8][4];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
-        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
-    }
+        for (int nt = 0; nt < D / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
 
-    // ---------------------------------------------- merge the four warps --
-    consumer_sync();   // every consumer finished reading the ring
-    float *red_o = reinterpret_cast<float *>(smem);                       // [warp][16][D]
-    float *red_ml = red_o + kConsumerWarps * 16 * D;                      // [warp][16][2]
+        for (int t = 0; t < it.ntiles; ++t, ++gt) {
+            const int st = gt % C::kStages;
+            const bool landed = ok && mbar_wait(smem_u32(full + st), (gt / C::kStages) & 1, a.dev_error);
+            if (!__all_sync(0xffffffffu, landed)) ok = false;
+            const uint32_t kbase = ring + st * C::kStageBytes;
+            const uint32_t vbase = kbase + C::kKvBytes;
+            const int tok0 = it.t_begin + t * kTile + warp * 16;   // first token of this warp's slice
+
+            // S = Q K^T over this warp's 16 tokens (two n-tiles of 8 tokens)
+            float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int g = g0 + r * 8;
-        if (g < G) {
-            float *dst = red_o + (warp * 16 + g) * D;
-#pragma unroll
-            for (int nt = 0; nt < D / 8; ++nt) {
-                dst[nt * 8 + c2] = o[nt][2 * r];
-                dst[nt * 8 + c2 + 1] = o[nt][2 * r + 1];
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const int trow = warp * 16 + (mi >> 1) * 8 + mr;
+                const int dch = ks * 2 + (mi & 1);
+                uint32_t b0n0, b1n0, b0n1, b1n1;
+                ldmatrix_x4(kbase + (dch >> 3) * kHalfBytes + swz128(trow, dch & 7), b0n0, b1n0, b0n1, b1n1);
+                mma_bf16_16816(sc[0], qa[ks], b0n0, b1n0);
+                mma_bf16_16816(sc[1], qa[ks], b0n1, b1n1);
             }
-            if ((lane & 3) == 0) {
-                red_ml[(warp * 16 + g) * 2] = m_run[r];
-                red_ml[(warp * 16 + g) * 2 + 1] = l_run[r];
+
+            // scale into log2 units and select out positions past the end
+            const bool partial = tok0 + 16 > it.t_end;
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int tok = tok0 + n * 8 + c2 + (e & 1);
+                    const float v = sc[n][e] * a.scale_log2;
+                    sc[n][e] = (!partial || tok < it.t_end) ? v : -INFINITY;
+                }
+
+            // online softmax (rows g0 and g0 + 8)
+            float mx[2];
+            mx[0] = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+            mx[1] = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+                mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+            }
+            float corr[2], ref[2];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const float m_new = fmaxf(m_run[r], mx[r]);
+                ref[r] = m_new == -INFINITY ? 0.f : m_new;
+                corr[r] = fast_exp2(m_run[r] - ref[r]);
+                m_run[r] = m_new;
+            }
+            float p[2][4];
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) p[n][e] = fast_exp2(sc[n][e] - ref[e >> 1]);
+            l_run[0] = l_run[0] * corr[0] + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
+            l_run[1] = l_run[1] * corr[1] + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
+            if (!__all_sync(0xffffffffu, corr[0] == 1.f && corr[1] == 1.f)) {
+#pragma unroll
+                for (int nt = 0; nt < D / 8; ++nt) {
+                    o[nt][0] *= corr[0];
+                    o[nt][1] *= corr[0];
+                    o[nt][2] *= corr[1];
+                    o[nt][3] *= corr[1];
+                }
+            }
+            uint32_t pa[4];
+            pa[0] = pack_bf16(p[0][0], p[0][1]);
+            pa[1] = pack_bf16(p[0][2], p[0][3]);
+            pa[2] = pack_bf16(p[1][0], p[1][1]);
+            pa[3] = pack_bf16(p[1][2], p[1][3]);
+
+            // V fragments hold tokens tok0 + c2 + {0,1} (b0) and tok0 + 8 + c2 + {0,1} (b1)
+            uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
+            if (partial) {
+                vm0 = (tok0 + c2 < it.t_end ? 0x0000ffffu : 0u) | (tok0 + c2 + 1 < it.t_end ? 0xffff0000u : 0u);
+                vm1 = (tok0 + 8 + c2 < it.t_end ? 0x0000ffffu : 0u) | (tok0 + 9 + c2 < it.t_end ? 0xffff0000u : 0u);
+            }
+#pragma unroll
+            for (int jp = 0; jp < D / 16; ++jp) {
+                const int trow = warp * 16 + (mi & 1) * 8 + mr;
+                const int dch = jp * 2 + (mi >> 1);
+                uint32_t b0a, b1a, b0b, b1b;
+                ldmatrix_x4_trans(vbase + (dch >> 3) * kHalfBytes + swz128(trow, dch & 7), b0a, b1a, b0b, b1b);
+                b0a &= vm0;
+                b1a &= vm1;
+                b0b &= vm0;
+                b1b &= vm1;
+                mma_bf16_16816(o[2 * jp], pa, b0a, b1a);
+                mma_bf16_16816(o[2 * jp + 1], pa, b0b, b1b);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(empty + st));
+        }
+
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
+            l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+        }
+        // ------------------------------------------ merge the four warps --
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int g = g0 + r * 8;
+            if (g < G) {
+                float *dst = red_o + (warp * G + g) * D;
+#pragma unroll
+                for (int nt = 0; nt < D / 8; ++nt) {
+                    dst[nt * 8 + c2] = o[nt][2 * r];
+                    dst[nt * 8 + c2 + 1] = o[nt][2 * r + 1];
+                }
+                if ((lane & 3) == 0) {
+                    red_ml[(warp * G + g) * 2] = m_run[r];
+                    red_ml[(warp * G + g) * 2 + 1] = l_run[r];
+                }
             }
         }
-    }
-    consumer_sync();
-    if (!ok) return;
-
-    const bool single = a.plan.max_splits == 1;
-    for (int e = threadIdx.x; e < G * D; e += kConsumerWarps * 32) {
-        const int g = e / D, d = e % D;
-        float mt = -INFINITY;
+        consumer_sync();
+        for (int e = threadIdx.x; e < G * D; e += kConsumerWarps * 32) {
+            const int g = e / D, d = e % D;
+            float mt = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) mt = fmaxf(mt, red_ml[(w * 16 + g) * 2]);
-        float lt = 0.f, ot = 0.f;
+            for (int w = 0; w < kConsumerWarps; ++w) mt = fmaxf(mt, red_ml[(w * G + g) * 2]);
+            float lt = 0.f, ot = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-            const float mw = red_ml[(w * 16 + g) * 2];
-            const float f = mw == -INFINITY ? 0.f : fast_exp2(mw - mt);
-            lt += f * red_ml[(w * 16 + g) * 2 + 1];
-            ot += f * red_o[(w * 16 + g) * D + d];
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float mw = red_ml[(w * G + g) * 2];
+                const float f = mw == -INFINITY ? 0.f : fast_exp2(mw - mt);
+                lt += f * red_ml[(w * G + g) * 2 + 1];
+                ot += f * red_o[(w * G + g) * D + d];
+            }
+            const int h = it.kvh * G + g;
+            if (single) {
+                static_cast<__nv_bfloat16 *>(a.out)[((int64_t)it.s * a.num_q_heads + h) * D + d] =
+                    __float2bfloat16_rn(ot / lt);
+            } else {
+                const int64_t pi = ((int64_t)it.s * a.num_q_heads + h) * a.plan.max_splits + it.split;
+                a.part_o[pi * D + d] = ot / lt;
+                if (d == 0) a.part_lse[pi] = mt + __log2f(lt);
+            }
         }
-        const int h = kvh * G + g;
-        if (single) {
-            static_cast<__nv_bfloat16 *>(a.out)[((int64_t)s * a.num_q_heads + h) * D + d] = __float2bfloat16_rn(ot / lt);
-        } else {
-            const int64_t pi = ((int64_t)s * a.num_q_heads + h) * a.plan.max_splits + split;
-            a.part_o[pi * D + d] = ot / lt;
-            if (d == 0) a.part_lse[pi] = mt + __log2f(lt);
-        }
+        consumer_sync();   // the merge area is free for the next item
     }
 }
 
@@ -337,19 +402,29 @@ template <int D>
 cudaError_t launch_decode_d(const DecodeArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                             cudaStream_t stream) {
     using C = DecodeCfg<D>;
-    static std::atomic<uint64_t> configured{0};   // one bit per device whose attribute is set
+    // attribute and occupancy per (device, G); G <= 16
+    static std::atomic<int> resident[64][17];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const uint64_t bit = uint64_t(1) << (dev & 63);
-    if (!(configured.load(std::memory_order_acquire) & bit)) {
+    const size_t smem = C::smem_bytes(a.group);
+    int per_sm = resident[dev & 63][a.group].load(std::memory_order_acquire);
+    if (per_sm == 0) {
         e = cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::kSmemBytes);
+                                 (int)C::smem_bytes(16));
         if (e != cudaSuccess) return e;
-        configured.fetch_or(bit, std::memory_order_acq_rel);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_split_kernel<D>, kThreads, smem);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) per_sm = 1;
+        resident[dev & 63][a.group].store(per_sm, std::memory_order_release);
     }
-    const dim3 grid((unsigned)a.plan.max_splits, (unsigned)a.num_kv_heads, (unsigned)a.batch);
-    decode_split_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tm_k, tm_v, a);
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int64_t n_items = (int64_t)a.plan.max_splits * a.batch * a.num_kv_heads;
+    const int64_t slots = (int64_t)per_sm * sms;
+    const int grid = (int)(n_items < slots ? n_items : slots);
+    decode_split_kernel<D><<<grid, kThreads, smem, stream>>>(tm_k, tm_v, a);
     e = cudaGetLastError();
     if (e != cudaSuccess || a.plan.max_splits == 1) return e;
 

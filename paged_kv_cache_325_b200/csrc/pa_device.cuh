@@ -98,6 +98,13 @@ PA_DEVICE void tma_load_3d(uint32_t dst, const CUtensorMap *map, int32_t c0, int
         : "memory");
 }
 
+// Non-tensor bulk copy global -> shared (both 16-byte aligned, bytes a multiple of 16), completion on `bar`.
+PA_DEVICE void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 // ------------------------------------------------------- warp-level MMA path --
 
 PA_DEVICE void ldmatrix_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {

@@ -345,6 +345,23 @@ def bench_secondary(args, device, pk, names):
                              "frac": uniq / tm / 1e9 / pk["hbm_gbs"], "bytes": "unique"}
             (tw,) = timer.run([dec_replay], steps, flush=False)
             r["decode_us_warm_l2"] = statistics.mean(tw) * 1e6
+            # the shared-prefix path: the 16 common blocks read once per KV head
+            P = case.shared_prefix_blocks
+            sws = pa.alloc_shared_prefix_workspace(b.q, case.num_kv_heads, b.mcl, case.block_size, P)
+
+            def shared():
+                pa.pa_decode_shared_prefix(b.out, b.q, b.k_cache, b.v_cache, b.bt, b.ctx, b.mcl, case.softmax_scale,
+                                           P, sws)
+
+            sh_replay, _g3 = capture(shared)
+            timer.run([sh_replay], 5)
+            (ts,) = timer.run([sh_replay], steps)
+            tsm = statistics.mean(ts)
+            r["shared_prefix_path"] = {
+                "decode_us": tsm * 1e6, "tokens_per_s": case.batch / tsm,
+                "kv_gbps_unique": case.kv_bytes_unique() / tsm / 1e9,
+                "roofline": {"bound": "hbm", "achieved": uniq / tsm / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": uniq / tsm / 1e9 / pk["hbm_gbs"], "bytes": "unique"}}
         out[name] = r
         del b, dec_replay, _g
         torch.cuda.empty_cache()

@@ -171,6 +171,36 @@ PA_API pa_status pa_decode_split(void *out, const void *q, const void *k_cache, 
                           void *stream);
 
 /*
+ * pa_decode_shared_prefix -- pa_decode for a batch whose sequences all start
+ * with the same num_shared_blocks physical blocks (a prefix-cache hit shared by
+ * the whole batch: block_table[s][0 .. num_shared_blocks) is the same for every
+ * s, as the BlockManager's whole-block prefix hashing produces, nano-vllm
+ * walkthrough, section five).  It computes exactly what pa_decode computes, but
+ * reads the shared blocks once per KV head instead of once per sequence:
+ *   1. all batch x G query rows of a KV head attend to the shared keys
+ *      together on the tensor cores (non-causal, the keys cut into chunks),
+ *      each chunk giving an fp32 partial and its log-sum-exp;
+ *   2. the split-KV decode covers each sequence's private tokens
+ *      [num_shared_blocks * block_size, context_lens[s]);
+ *   3. all partials of a (sequence, q-head) are merged by log-sum-exp.
+ * Every context_lens[s] must be >= num_shared_blocks * block_size (checked
+ * mode reports PA_DEVERR_CONTEXT_LEN; a table row whose first blocks differ
+ * from row 0's is reported as PA_DEVERR_BLOCK_ID).  The GQA group must divide
+ * 128.  Workspace: pa_decode_shared_prefix_workspace_size() bytes, 256-byte
+ * aligned, no initialisation needed.
+ */
+PA_API size_t pa_decode_shared_prefix_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                                     int32_t head_dim, int32_t max_context_len, int32_t block_size,
+                                                     int32_t num_shared_blocks);
+PA_API pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                         const int32_t *block_table, int32_t block_table_stride,
+                                         const int32_t *context_lens, int32_t batch, int32_t max_context_len,
+                                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t num_blocks, int32_t block_size, float softmax_scale,
+                                         int32_t num_shared_blocks, void *workspace, size_t workspace_bytes,
+                                         int32_t *dev_error, void *stream);
+
+/*
  * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
  * memory (no counterpart in the pages: it exists for integration, not for the
  * method).  Some hosts own every device allocation themselves -- a plugin

@@ -33,7 +33,8 @@ PA_DEVERR_SEQLENS = 0x8
 PA_DEVERR_TIMEOUT = 0x10
 
 __all__ = ["PagedAttnError", "load_library", "declared_symbols", "pa_store_kv", "pa_decode", "pa_decode_split",
-           "pa_decode_workspace_size", "pa_decode_split_workspace_size", "pa_decode_noalloc", "pa_prefill_varlen",
+           "pa_decode_workspace_size", "pa_decode_split_workspace_size", "pa_decode_noalloc",
+           "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size", "alloc_shared_prefix_workspace", "pa_prefill_varlen",
            "pa_prefill_workspace_size", "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
            "alloc_decode_workspace", "alloc_prefill_workspace"]
 
@@ -58,6 +59,10 @@ _SIGS = {
                                  _c_i32, _c_i32, _c_i32, _c_f32, _c_p, _c_sz, _c_p, _c_p]),
     "pa_decode_split": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_i32,
                                        _c_i32, _c_i32, _c_i32, _c_f32, _c_i32, _c_p, _c_sz, _c_p, _c_p]),
+    "pa_decode_shared_prefix_workspace_size": (_c_sz, [_c_i32] * 7),
+    "pa_decode_shared_prefix": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_i32, _c_i32, _c_i32,
+                                               _c_i32, _c_i32, _c_i32, _c_i32, _c_f32, _c_i32, _c_p, _c_sz, _c_p,
+                                               _c_p]),
     "pa_decode_noalloc_max_scratch_bytes": (_c_sz, []),
     "pa_decode_noalloc": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_i32,
                                          _c_i32, _c_i32, _c_i32, _c_f32, _c_p, _c_p]),
@@ -228,6 +233,32 @@ def pa_decode_split(out, q, k_cache, v_cache, block_table, context_lens, max_con
     """pa_decode with an explicit number of context splits (0 = automatic)."""
     pa_decode(out, q, k_cache, v_cache, block_table, context_lens, max_context_len, softmax_scale,
               workspace=workspace, dev_error=dev_error, stream=stream, num_splits=num_splits)
+
+
+def pa_decode_shared_prefix_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, block_size,
+                                           num_shared_blocks) -> int:
+    return int(load_library().pa_decode_shared_prefix_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
+                                                                      max_context_len, block_size, num_shared_blocks))
+
+
+def alloc_shared_prefix_workspace(q, num_kv_heads, max_context_len, block_size, num_shared_blocks):
+    import torch
+    batch, Hq, D = q.shape
+    n = pa_decode_shared_prefix_workspace_size(batch, Hq, num_kv_heads, D, max_context_len, block_size,
+                                               num_shared_blocks)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+
+
+def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_table, context_lens, max_context_len, softmax_scale,
+                            num_shared_blocks, workspace, dev_error=None, stream=None):
+    """Decode for a batch whose block tables all start with the same num_shared_blocks blocks."""
+    nb, B, Hkv, D, batch, Hq, dev = _decode_args(out, q, k_cache, v_cache, block_table, context_lens)
+    _need(workspace, "workspace", None, dev)
+    _check(load_library().pa_decode_shared_prefix(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
+        _ptr(context_lens), batch, int(max_context_len), Hq, Hkv, D, nb, B, float(softmax_scale),
+        int(num_shared_blocks), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _opt_err(dev_error, dev), _stream(q, stream)))
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_table, context_lens, max_context_len, softmax_scale,

@@ -77,11 +77,12 @@ __device__ __forceinline__ DecItem dec_item(const DecodeArgs &a, int i, bool rep
     it.kvh = r % a.num_kv_heads;
     it.valid = 0;
     const int ctx = __ldg(a.context_lens + it.s);
-    if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size) {
+    if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size ||
+        ctx < a.t_offset) {
         if (report_bad && it.split == 0 && it.kvh == 0) report(a.dev_error, PA_DEVERR_CONTEXT_LEN);
         return it;
     }
-    it.t_begin = it.split * a.plan.chunk;
+    it.t_begin = a.t_offset + it.split * a.plan.chunk;
     if (it.t_begin >= ctx) return it;            // this split lies past the end of the context
     it.t_end = min(ctx, it.t_begin + a.plan.chunk);
     it.ntiles = (it.t_end - it.t_begin + kTile - 1) / kTile;
@@ -144,6 +145,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                           qbytes, smem_u32(qfull + qs));
                 ++nqi;
                 const int32_t *bt = a.block_table + (int64_t)it.s * a.bt_stride;
+                if (a.dev_error && a.shared_blocks > 0 && it.split == 0 && it.kvh == 0)
+                    for (int b = 0; b < a.shared_blocks; ++b)
+                        if (__ldg(bt + b) != __ldg(a.block_table + b)) report(a.dev_error, PA_DEVERR_BLOCK_ID);
                 for (int t = 0; t < it.ntiles; ++t, ++gt) {
                     const int st = gt % C::kStages;
                     if (gt >= (uint32_t)C::kStages &&
@@ -190,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int g0 = lane >> 2;             // accumulator rows g0 and g0 + 8
     const int c2 = (lane & 3) * 2;        // accumulator columns c2, c2 + 1
     const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: matrix index / row this lane addresses
-    const bool single = a.plan.max_splits == 1;
+    const bool single = a.plan.max_splits == 1 && !a.force_partial;
     uint32_t gt = 0, nqi = 0;
     bool ok = true;
     for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
@@ -367,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 static_cast<__nv_bfloat16 *>(a.out)[((int64_t)it.s * a.num_q_heads + h) * D + d] =
                     __float2bfloat16_rn(ot / lt);
             } else {
-                const int64_t pi = ((int64_t)it.s * a.num_q_heads + h) * a.plan.max_splits + it.split;
+                const int64_t pi = ((int64_t)it.s * a.num_q_heads + h) * a.part_slots + a.part_base + it.split;
                 a.part_o[pi * D + d] = ot / lt;
                 if (d == 0) a.part_lse[pi] = mt + __log2f(lt);
             }
@@ -383,14 +387,18 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
     const int h = blockIdx.x % a.num_q_heads;
     const int s = blockIdx.x / a.num_q_heads;
     const int ctx = __ldg(a.context_lens + s);
-    if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size) return;
-    const int nsplit = (ctx + a.plan.chunk - 1) / a.plan.chunk;
-    const int64_t base = ((int64_t)s * a.num_q_heads + h) * a.plan.max_splits;
+    if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size ||
+        ctx < a.t_offset)
+        return;
+    // partials: part_base slots written before this launch (shared-prefix chunks), then the splits
+    const int nsplit = (ctx - a.t_offset + a.plan.chunk - 1) / a.plan.chunk;
+    const int n = a.part_base + nsplit;
+    const int64_t base = ((int64_t)s * a.num_q_heads + h) * a.part_slots;
     float mt = -INFINITY;
-    for (int i = 0; i < nsplit; ++i) mt = fmaxf(mt, a.part_lse[base + i]);
+    for (int i = 0; i < n; ++i) mt = fmaxf(mt, a.part_lse[base + i]);
     float den = 0.f, num = 0.f;
     const int d = threadIdx.x;
-    for (int i = 0; i < nsplit; ++i) {
+    for (int i = 0; i < n; ++i) {
         const float w = fast_exp2(a.part_lse[base + i] - mt);
         den += w;
         num += w * a.part_o[(base + i) * D + d];
@@ -426,7 +434,7 @@ cudaError_t launch_decode_d(const DecodeArgs &a, const CUtensorMap &tm_k, const 
     const int grid = (int)(n_items < slots ? n_items : slots);
     decode_split_kernel<D><<<grid, kThreads, smem, stream>>>(tm_k, tm_v, a);
     e = cudaGetLastError();
-    if (e != cudaSuccess || a.plan.max_splits == 1) return e;
+    if (e != cudaSuccess || (a.plan.max_splits == 1 && !a.force_partial)) return e;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.batch * a.num_q_heads));
@@ -468,9 +476,10 @@ DecodePlan plan_decode(int32_t batch, int32_t num_kv_heads, int32_t max_context_
     return p;
 }
 
-size_t decode_workspace_bytes(const DecodePlan &plan, int32_t batch, int32_t num_q_heads, int32_t head_dim) {
-    if (plan.max_splits <= 1) return 0;
-    const size_t n = (size_t)batch * num_q_heads * plan.max_splits;
+size_t decode_workspace_bytes(const DecodePlan &plan, int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                              int32_t extra_slots) {
+    if (plan.max_splits <= 1 && extra_slots == 0) return 0;
+    const size_t n = (size_t)batch * num_q_heads * (plan.max_splits + extra_slots);
     const size_t o_bytes = (n * head_dim * sizeof(float) + 255) / 256 * 256;
     return o_bytes + n * sizeof(float);
 }

@@ -223,6 +223,11 @@ static pa_status decode_impl(void *out, const void *q, const void *k_cache, cons
     a.box_tokens = block_size < pa::kDecodeTileTokens ? block_size : pa::kDecodeTileTokens;
     a.max_context_len = max_context_len;
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
+    a.part_slots = a.plan.max_splits;
+    a.part_base = 0;
+    a.t_offset = 0;
+    a.force_partial = 0;
+    a.shared_blocks = 0;
 
     CUtensorMap tm_k, tm_v;
     const int64_t rows = (int64_t)num_blocks * block_size;
@@ -261,6 +266,172 @@ pa_status pa_decode_split(void *out, const void *q, const void *k_cache, const v
     return decode_impl(out, q, k_cache, v_cache, block_table, block_table_stride, context_lens, batch,
                        max_context_len, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, softmax_scale,
                        num_splits, workspace, workspace_bytes, dev_error, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Work split of the shared-prefix decode: the prefix keys are cut into chunks so that the prefix phase
+// has about two work units per SM; the private suffixes use the ordinary decode split.
+struct SharedPlan {
+    pa::DecodePlan dplan;
+    int32_t nchunks, key_chunk, ranks, slots;
+    size_t plan_bytes, o_bytes, lse_bytes, total;
+};
+
+SharedPlan plan_shared(int32_t batch, int32_t Hq, int32_t Hkv, int32_t D, int32_t max_ctx, int32_t B, int32_t P,
+                       int sms) {
+    SharedPlan sp;
+    const int32_t G = Hq / Hkv, TQ = 128 / G;
+    const int64_t nprefix = (int64_t)P * B;
+    sp.ranks = (batch + 2 * TQ - 1) / (2 * TQ);
+    const int64_t per_chunk_units = (int64_t)sp.ranks * Hkv;
+    int64_t nch = (2 * (int64_t)sms + per_chunk_units - 1) / per_chunk_units;
+    const int64_t max_ch = (nprefix + 127) / 128;
+    if (nch < 1) nch = 1;
+    if (nch > max_ch) nch = max_ch;
+    int64_t kc = (nprefix + nch - 1) / nch;
+    kc = (kc + 127) / 128 * 128;
+    sp.key_chunk = (int32_t)kc;
+    sp.nchunks = (int32_t)((nprefix + kc - 1) / kc);
+    const int32_t suffix = max_ctx - (int32_t)nprefix > 0 ? max_ctx - (int32_t)nprefix : 1;
+    sp.dplan = pa::plan_decode(batch, Hkv, suffix, 0, sms);
+    sp.slots = sp.nchunks + sp.dplan.max_splits;
+    auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
+    sp.plan_bytes = r256(pa::prefill_workspace_bytes(1, batch, G, Hkv, sp.nchunks));
+    sp.o_bytes = r256((size_t)batch * Hq * sp.slots * D * sizeof(float));
+    sp.lse_bytes = r256((size_t)batch * Hq * sp.slots * sizeof(float));
+    sp.total = sp.plan_bytes + sp.o_bytes + sp.lse_bytes;
+    return sp;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pa_decode_shared_prefix_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                              int32_t head_dim, int32_t max_context_len, int32_t block_size,
+                                              int32_t num_shared_blocks) {
+    if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || head_dim <= 0 ||
+        max_context_len <= 0 || block_size <= 0 || num_shared_blocks <= 0 ||
+        128 % (num_q_heads / num_kv_heads) != 0)
+        return 0;
+    return plan_shared(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, block_size, num_shared_blocks,
+                       num_sms_current())
+        .total;
+}
+
+pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                  const int32_t *block_table, int32_t block_table_stride,
+                                  const int32_t *context_lens, int32_t batch, int32_t max_context_len,
+                                  int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                                  int32_t block_size, float softmax_scale, int32_t num_shared_blocks,
+                                  void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream) {
+    if (batch < 0) return fail(PA_ERR_INVALID_ARG, "batch < 0");
+    pa_status st = check_cache_shape(num_blocks, block_size, num_kv_heads, head_dim);
+    if (st != PA_OK) return st;
+    if ((st = check_heads(num_q_heads, num_kv_heads)) != PA_OK) return st;
+    const int32_t G = num_q_heads / num_kv_heads;
+    if (128 % G != 0) return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode needs a GQA group that divides 128");
+    if (!(softmax_scale > 0.f) || !isfinite(softmax_scale))
+        return fail(PA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if (batch == 0) return ok();
+    if (max_context_len < 1 || block_table_stride < 1) return fail(PA_ERR_INVALID_ARG, "bad max_context_len or stride");
+    if (num_shared_blocks < 1 || num_shared_blocks > block_table_stride ||
+        (int64_t)num_shared_blocks * block_size > max_context_len)
+        return fail(PA_ERR_INVALID_ARG, "num_shared_blocks must be in [1, stride] and cover at most max_context_len");
+    if (batch > 65535 * 64) return fail(PA_ERR_UNSUPPORTED, "batch too large");
+    if (!out || !q || !k_cache || !v_cache || !block_table || !context_lens)
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_table, 4) || !aligned(context_lens, 4) || (dev_error && !aligned(dev_error, 4)))
+        return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
+    const int sms = num_sms_current();
+    const SharedPlan sp = plan_shared(batch, num_q_heads, num_kv_heads, head_dim, max_context_len, block_size,
+                                      num_shared_blocks, sms);
+    if (!workspace || workspace_bytes < sp.total)
+        return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", sp.total,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (!aligned(workspace, 256)) return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    char *ws = static_cast<char *>(workspace);
+    float *part_o = reinterpret_cast<float *>(ws + sp.plan_bytes);
+    float *part_lse = reinterpret_cast<float *>(ws + sp.plan_bytes + sp.o_bytes);
+    const int64_t rows = (int64_t)num_blocks * block_size;
+    const int32_t nprefix = num_shared_blocks * block_size;
+    cudaStream_t str = static_cast<cudaStream_t>(stream);
+
+    // 1. prefix: every query of the batch against the shared blocks (row 0 of the table), non-causal,
+    //    as one prefill "sequence" of `batch` query rows; fp32 partials per key chunk
+    pa::PrefillArgs pf = {};
+    pf.q = q;
+    pf.cu_q = pf.cu_k = nullptr;
+    pf.block_table = block_table;
+    pf.dev_error = dev_error;
+    pf.bt_stride = block_table_stride;
+    pf.batch = 1;
+    pf.num_q_heads = num_q_heads;
+    pf.num_kv_heads = num_kv_heads;
+    pf.group = G;
+    pf.head_dim = head_dim;
+    pf.num_blocks = num_blocks;
+    pf.block_size = block_size;
+    pf.box_tokens = block_size < 128 ? block_size : 128;
+    pf.max_seqlen_q = batch;
+    pf.max_seqlen_k = nprefix;
+    pf.causal = 0;
+    pf.total_q = batch;
+    pf.ranks = sp.ranks;
+    pf.workspace = ws;
+    pf.scale_log2 = softmax_scale * 1.4426950408889634f;
+    pf.single_n_new = batch;
+    pf.single_n_k = nprefix;
+    pf.key_chunk = sp.key_chunk;
+    pf.nchunks = sp.nchunks;
+    pf.part_o = part_o;
+    pf.part_lse = part_lse;
+    pf.part_slots = sp.slots;
+    pf.part_base = 0;
+    CUtensorMap tq, tk, tv;
+    if ((st = encode_rows(&tq, q, batch, num_q_heads, head_dim, G, 128 / G)) != PA_OK) return st;
+    if ((st = encode_rows(&tk, k_cache, rows, num_kv_heads, head_dim, 1, pf.box_tokens)) != PA_OK) return st;
+    if ((st = encode_rows(&tv, v_cache, rows, num_kv_heads, head_dim, 1, pf.box_tokens)) != PA_OK) return st;
+    cudaError_t e = pa::launch_prefill(pf, tq, tk, tv, str);
+    if (e != cudaSuccess) return cuda_fail(e, "shared-prefix kernel launch");
+
+    // 2. private suffixes: split-KV decode from token nprefix on, partials after the prefix chunks;
+    // 3. the combine kernel merges all partials of each (sequence, q-head)
+    pa::DecodeArgs da;
+    da.plan = sp.dplan;
+    da.out = out;
+    da.q = q;
+    da.block_table = block_table;
+    da.context_lens = context_lens;
+    da.dev_error = dev_error;
+    da.part_o = part_o;
+    da.part_lse = part_lse;
+    da.bt_stride = block_table_stride;
+    da.batch = batch;
+    da.num_q_heads = num_q_heads;
+    da.num_kv_heads = num_kv_heads;
+    da.group = G;
+    da.head_dim = head_dim;
+    da.num_blocks = num_blocks;
+    da.block_size = block_size;
+    da.box_tokens = block_size < pa::kDecodeTileTokens ? block_size : pa::kDecodeTileTokens;
+    da.max_context_len = max_context_len;
+    da.scale_log2 = pf.scale_log2;
+    da.part_slots = sp.slots;
+    da.part_base = sp.nchunks;
+    da.t_offset = nprefix;
+    da.force_partial = 1;
+    da.shared_blocks = num_shared_blocks;
+    CUtensorMap dk, dv;
+    if ((st = encode_rows(&dk, k_cache, rows, num_kv_heads, head_dim, 1, da.box_tokens)) != PA_OK) return st;
+    if ((st = encode_rows(&dv, v_cache, rows, num_kv_heads, head_dim, 1, da.box_tokens)) != PA_OK) return st;
+    e = pa::launch_decode(da, dk, dv, str);
+    if (e != cudaSuccess) return cuda_fail(e, "shared-prefix suffix decode launch");
+    return ok();
 }
 
 size_t pa_prefill_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t num_q_heads, int32_t num_kv_heads,
@@ -328,6 +499,11 @@ pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const voi
     a.total_q = total_q;
     a.ranks = (max_seqlen_q + 2 * (128 / a.group) - 1) / (2 * (128 / a.group));
     a.workspace = workspace;
+    a.single_n_new = a.single_n_k = 0;
+    a.key_chunk = 0;
+    a.nchunks = 1;
+    a.part_o = a.part_lse = nullptr;
+    a.part_slots = a.part_base = 0;
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
 
     CUtensorMap tm_k, tm_v;

@@ -32,7 +32,8 @@ struct DecodePlan {
 };
 DecodePlan plan_decode(int32_t batch, int32_t num_kv_heads, int32_t max_context_len, int32_t num_splits,
                        int32_t num_sms);
-size_t decode_workspace_bytes(const DecodePlan &plan, int32_t batch, int32_t num_q_heads, int32_t head_dim);
+size_t decode_workspace_bytes(const DecodePlan &plan, int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                              int32_t extra_slots = 0);
 
 struct DecodeArgs {
     void *out;
@@ -46,6 +47,11 @@ struct DecodeArgs {
     int32_t num_blocks, block_size, box_tokens, max_context_len;
     DecodePlan plan;
     float scale_log2;
+    // the partials of (sequence s, q-head h) sit at slots [part_base, part_base + splits) of part_slots
+    int32_t part_slots, part_base;
+    int32_t t_offset;        // the split ranges start at this token (shared-prefix decode: P * block_size)
+    int32_t force_partial;   // write partials (and run the combine) even with one split
+    int32_t shared_blocks;   // checked mode: block_table[s][0..shared_blocks) must equal row 0's
 };
 cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                           cudaStream_t stream);
@@ -61,8 +67,14 @@ struct PrefillArgs {
     int32_t ranks;              // pairs of Q tiles of the longest sequence
     void *workspace;            // unit table + hand-out counter (prefill_workspace_bytes)
     float scale_log2;
+    // --- used by the shared-prefix decode (zero / NULL for pa_prefill_varlen) ---
+    int32_t single_n_new, single_n_k;   // cu_q == NULL: one sequence with these sizes
+    int32_t key_chunk, nchunks;         // non-causal: split the keys into chunks of key_chunk (0: one chunk)
+    float *part_o, *part_lse;           // non-NULL: write fp32 partials [row, head, part_slots, D] + lse
+    int32_t part_slots, part_base;      // partial slots per (row, head); first slot used by chunk 0
 };
-size_t prefill_workspace_bytes(int32_t batch, int32_t max_seqlen_q, int32_t group, int32_t num_kv_heads);
+size_t prefill_workspace_bytes(int32_t batch, int32_t max_seqlen_q, int32_t group, int32_t num_kv_heads,
+                               int32_t nchunks = 1);
 constexpr int32_t kPrefillMaxBatch = 6144;   // the planning kernel keeps 2 ints per sequence in shared memory
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                            const CUtensorMap &tm_v, cudaStream_t stream);

@@ -79,9 +79,10 @@ struct Unit {                 // 16 words; copied through the shared-memory unit
     int s, kvh;
     int q0;          // row of the sequence's first new token in q / out
     int n_new, n_k, c;
+    int kbeg;        // first key of the unit's key range (a multiple of 128)
+    int chunk;       // key chunk index (0 unless the key range is split)
     int tok0[2];     // first new token of tile A / B (relative to the sequence)
-    int nq[2];       // tokens in tile A / B (0: tile absent)
-    int kend[2];     // keys [0, kend) visible to some row of the tile
+    int kend[2];     // keys [kbeg, kend) visible to some row of the tile (kend = kbeg: tile absent)
     int nt[2];       // key tiles of tile A / B
     int nk;          // key tiles loaded for the unit
 };
@@ -89,6 +90,13 @@ static_assert(sizeof(Unit) == 64, "Unit is copied as 16 words");
 
 // Geometry of one sequence; false when its cu_seqlens are inconsistent.
 __device__ __forceinline__ bool seq_geometry(const PrefillArgs &a, int s, int &q0, int &n_new, int &n_k) {
+    if (!a.cu_q) {                    // one sequence given by scalars
+        q0 = 0;
+        n_new = a.single_n_new;
+        n_k = a.single_n_k;
+        return s == 0 && n_new >= 0 && n_k >= 1 && n_new <= a.total_q && n_new <= a.max_seqlen_q &&
+               n_k <= a.max_seqlen_k && (int64_t)n_k <= (int64_t)a.bt_stride * a.block_size;
+    }
     q0 = a.cu_q[s];
     const int q1 = a.cu_q[s + 1];
     const int k0 = a.cu_k[s], k1 = a.cu_k[s + 1];
@@ -126,6 +134,7 @@ __device__ __forceinline__ Unit unit_from_record(const PrefillArgs &a, int4 rec,
     U.s = rec.x;
     U.kvh = rec.y;
     const int r = rec.z;
+    U.chunk = rec.w;
     if (!geo.w) return U;
     U.q0 = geo.x;
     U.n_new = geo.y;
@@ -134,11 +143,14 @@ __device__ __forceinline__ Unit unit_from_record(const PrefillArgs &a, int4 rec,
     const int npairs = (U.n_new + 2 * TQ - 1) / (2 * TQ);
     if (r >= npairs) return U;
     const int p = npairs - 1 - r;
+    // key range: the whole context, or one chunk of it when a non-causal call splits the keys
+    U.kbeg = a.key_chunk > 0 ? U.chunk * a.key_chunk : 0;
+    const int kmax = a.key_chunk > 0 ? min(U.n_k, U.kbeg + a.key_chunk) : U.n_k;
     for (int x = 0; x < 2; ++x) {
         U.tok0[x] = (2 * p + x) * TQ;
-        U.nq[x] = max(0, min(TQ, U.n_new - U.tok0[x]));
-        U.kend[x] = U.nq[x] == 0 ? 0 : (a.causal ? U.c + U.tok0[x] + U.nq[x] : U.n_k);
-        U.nt[x] = (U.kend[x] + kN - 1) / kN;
+        const int nq = max(0, min(TQ, U.n_new - U.tok0[x]));
+        U.kend[x] = nq == 0 ? U.kbeg : (a.causal ? U.c + U.tok0[x] + nq : kmax);
+        U.nt[x] = (U.kend[x] - U.kbeg + kN - 1) / kN;
     }
     U.nk = max(U.nt[0], U.nt[1]);
     U.valid = 1;
@@ -191,7 +203,7 @@ __global__ void __launch_bounds__(kPlanThreads)
             const int mid = (lo + hi) >> 1;
             if (nps[mid] > r) lo = mid + 1; else hi = mid;
         }
-        local += lo * a.num_kv_heads;
+        local += lo * a.num_kv_heads * a.nchunks;
     }
     // exclusive block scan of `local`
     const int lane = tid & 31, wid = tid >> 5;
@@ -221,7 +233,7 @@ __global__ void __launch_bounds__(kPlanThreads)
             const int mid = (lo + hi) >> 1;
             if (nps[mid] > r) lo = mid + 1; else hi = mid;
         }
-        run += lo * a.num_kv_heads;
+        run += lo * a.num_kv_heads * a.nchunks;
     }
     if (r1 == R && r0 < R) prefix[R] = run;
     if (R == 0 && tid == 0) prefix[0] = 0;
@@ -234,7 +246,8 @@ __global__ void __launch_bounds__(kPlanThreads)
             if (prefix[mid] <= u) lo = mid; else hi = mid;
         }
         const int i = u - prefix[lo];
-        units[u] = make_int4(order[i / a.num_kv_heads], i % a.num_kv_heads, lo, 0);
+        const int per_seq = a.num_kv_heads * a.nchunks;
+        units[u] = make_int4(order[i / per_seq], (i % per_seq) / a.nchunks, lo, i % a.nchunks);
     }
     if (tid == 0) {
         w[0] = 0;                                 // hand-out counter
@@ -391,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int chunk = -32, ids = 0;            // block_table[chunk + lane] lives in `ids` of that lane
                 if (ok && U.nk > 0) ++nvlast;
                 for (int j = 0; j < U.nk && ok; ++j) {
-                    const int key0 = j * kN;
+                    const int key0 = U.kbeg + j * kN;
                     const int nbox = (min(kN, kend - key0) + box - 1) / box;
                     const int last_blk = (key0 + (nbox - 1) * box) / B;
                     if (last_blk >= chunk + 32) {
@@ -562,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             L += 2 * U.nk;
             if (!mbar_wait(smem_u32(vlast_full + (nfx & 1)), (nfx >> 1) & 1, a.dev_error)) break;
             ++nfx;
-            const int valid = max(U.kend[0], U.kend[1]) - (U.nk - 1) * kN;
+            const int valid = max(U.kend[0], U.kend[1]) - (U.kbeg + (U.nk - 1) * kN);
             if (valid < kN) {
                 const uint32_t vs = ring + (vidx % C::kSlots) * C::kTileBytes;
                 for (int e = lane; e < (kN - valid) * C::kHalves * 8; e += 32) {
@@ -590,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!U.valid || U.nt[x] == 0) continue;
             const int t = U.tok0[x] + r / G;              // this row's new-token index
             int lim = a.causal ? U.c + t : U.n_k - 1;      // last visible key
-            if (lim > U.n_k - 1) lim = U.n_k - 1;          // rows past n_new never see past the keys
+            if (lim > U.kend[x] - 1) lim = U.kend[x] - 1;  // never past the unit's key range
             float m_ref = -INFINITY, l = 0.f;
             bool ok = true;
             for (int j = 0; j < U.nt[x]; ++j) {
@@ -601,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) tmem_ld32(lane_base + col_s(x) + q * 32, sr[q]);
                 tc_wait_ld();
-                const int thr = lim - j * kN;              // keys e <= thr are visible
+                const int thr = lim - (U.kbeg + j * kN);   // keys e <= thr are visible
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 if (thr >= kN - 1) {
 #pragma unroll
@@ -672,7 +685,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q = 0; q < D / 32; ++q) tmem_ld32(lane_base + col_o(x) + q * 32, o[q]);
             tc_wait_ld();
-            if (store) {
+            if (store && a.part_o) {
+                // partial result of this key chunk: fp32 O / l and its log-sum-exp (log2 units), to be merged
+                // with the other partials of the same (query, head)
+                const int64_t pi = ((int64_t)(U.q0 + t) * a.num_q_heads + (int64_t)U.kvh * G + r % G) * a.part_slots +
+                                   a.part_base + U.chunk;
+                float4 *po = reinterpret_cast<float4 *>(a.part_o + pi * D);
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q)
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        po[(q * 32 + e) / 4] = make_float4(__uint_as_float(o[q][e]) * inv, __uint_as_float(o[q][e + 1]) * inv,
+                                                           __uint_as_float(o[q][e + 2]) * inv, __uint_as_float(o[q][e + 3]) * inv);
+                a.part_lse[pi] = m_ref + __log2f(l);
+            } else if (store) {
 #pragma unroll
                 for (int q = 0; q < D / 32; ++q)
 #pragma unroll
@@ -725,7 +751,7 @@ cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &tm_q, cons
     prefill_plan_kernel<<<1, kPlanThreads, plan_smem, stream>>>(a, a.ranks, 2 * TQ);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int64_t max_units = (int64_t)a.ranks * a.batch * a.num_kv_heads;
+    const int64_t max_units = (int64_t)a.ranks * a.batch * a.num_kv_heads * a.nchunks;
     const int grid = (int)(max_units < num_sms() ? max_units : num_sms());
     if (grid <= 0) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};
@@ -743,11 +769,12 @@ cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &tm_q, cons
 
 }  // namespace
 
-size_t prefill_workspace_bytes(int32_t batch, int32_t max_seqlen_q, int32_t group, int32_t num_kv_heads) {
+size_t prefill_workspace_bytes(int32_t batch, int32_t max_seqlen_q, int32_t group, int32_t num_kv_heads,
+                               int32_t nchunks) {
     const int32_t TQ = kM / group;
     const int64_t R = ((int64_t)max_seqlen_q + 2 * TQ - 1) / (2 * TQ);
     const PlanLayout lay = plan_layout((int32_t)R, batch);
-    const size_t words = (size_t)lay.units + (size_t)4 * R * batch * num_kv_heads;
+    const size_t words = (size_t)lay.units + (size_t)4 * R * batch * num_kv_heads * nchunks;
     return (words * sizeof(int32_t) + 255) / 256 * 256;
 }
 

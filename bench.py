@@ -365,6 +365,8 @@ def bench_secondary(args, device, pk, names):
         out[name] = r
         del b, dec_replay, _g
         torch.cuda.empty_cache()
+    if "block_size_sweep" in names:
+        out["block_size_sweep"] = block_size_sweep(device, pk, timer, steps)
     if "varlen_prefill" not in names:
         return out
     case = W.varlen_prefill(poison=False, keep_contiguous=False)
@@ -403,6 +405,49 @@ def bench_secondary(args, device, pk, names):
                      "traffic": recorded_traffic("prefill_varlen")},
     }
     return out
+
+
+def block_size_sweep(device, pk, timer, steps):
+    """Decode (Qwen3-0.6B-like shape) and varlen prefill at several block sizes: the same token
+    counts, more and smaller pages (more block-table reads, smaller TMA boxes)."""
+    import paged_kv_cache_325_b200 as pa
+    from paged_kv_cache_325_b200 import workloads as W
+    res = {"decode": {}, "prefill": {}}
+    ctx = np.random.Generator(np.random.PCG64(1002)).integers(100, 1025, size=64).astype(np.int32)
+    for B in (16, 32, 64, 128, 256):
+        case = W.make_decode_case(ctx, 16, 8, 128, B, seed=2002, poison=False, keep_contiguous=False)
+        b = DecodeBench(case, device)
+        b.store()
+        rep, _g = capture(b.decode)
+        timer.run([rep], 5)
+        (t,) = timer.run([rep], steps)
+        tm = statistics.mean(t)
+        res["decode"][str(B)] = {"decode_us": tm * 1e6, "kv_gbps": case.kv_bytes_read() / tm / 1e9,
+                                 "frac": b.alg_bytes_decode() / tm / 1e9 / pk["hbm_gbs"]}
+        del b, rep, _g
+    base = W.varlen_prefill(poison=False, keep_contiguous=False)
+    for B in (16, 64, 256):
+        c = W.make_prefill_case(base.prompt_lens, base.cached_lens, 32, 8, 128, B, seed=2005, poison=False,
+                                keep_contiguous=False)
+        kc, vc = c.k_cache.to(device), c.v_cache.to(device)
+        q = c.q.to(device)
+        o = torch.empty_like(q)
+        args = [torch.as_tensor(x).to(device) for x in (c.cu_seqlens_q, c.cu_seqlens_k, c.block_table)]
+        ws = pa.alloc_prefill_workspace(q, 8, c.batch, c.max_seqlen_q)
+        pa.pa_store_kv(c.k_new.to(device), c.v_new.to(device), torch.as_tensor(c.slot_mapping).to(device), kc, vc)
+
+        def pf():
+            pa.pa_prefill_varlen(o, q, kc, vc, args[0], args[1], c.max_seqlen_q, c.max_seqlen_k, args[2],
+                                 c.softmax_scale, workspace=ws)
+
+        rep, _g = capture(pf)
+        timer.run([rep], 5)
+        (t,) = timer.run([rep], steps)
+        tm = statistics.mean(t)
+        res["prefill"][str(B)] = {"prefill_us": tm * 1e6, "tflops": c.causal_flops() / tm / 1e12}
+        del rep, _g
+    torch.cuda.empty_cache()
+    return res
 
 
 def local_gpu_index(device):

@@ -6,8 +6,9 @@
 
 One step = one attention-layer call of the Qwen3-0.6B-like decode workload
 (batch 64, context lengths U[100, 1024], 16 q / 8 kv heads, head_dim 128,
-block_size 256): pa_store_kv of the 64 new K/V rows, then pa_decode (split
-kernel + combine).  `value` is decode tokens/s over all ranks (each rank runs
+block_size 256): the store of the 64 new K/V rows and the paged decode, in
+one launch (pa_store_kv_decode; the two-launch form, pa_store_kv then
+pa_decode, is timed beside it).  `value` is decode tokens/s over all ranks (each rank runs
 its own replica: the path shards by sequence with no exchange, so scaling is
 weak).  Inputs are resident in HBM; L2 is flushed (256 MiB write) before
 every timed step; each step is timed with CUDA events on the launching
@@ -43,7 +44,8 @@ if ROOT not in sys.path:
 METRIC = "paged decode tokens/s and KV HBM GB/s (% of B200 peak); prefill TFLOP/s"
 PRIMARY = "qwen3_0.6b_decode"
 PRIMARY_DESC = ("Qwen3-0.6B-like decode layer call: batch 64, context_lens U[100,1024], 16 q / 8 kv heads, "
-                "head_dim 128, block_size 256, shuffled blocks; pa_store_kv of 64 new rows + pa_decode")
+                "head_dim 128, block_size 256, shuffled blocks; store of the 64 new K/V rows + paged decode "
+                "(pa_store_kv_decode, one launch)")
 FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -243,8 +245,11 @@ class DecodeBench:
         self.pa.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.bt, self.ctx, self.mcl, c.softmax_scale,
                           workspace=self.ws)
 
-    def launches_per_step(self):
-        return 1 + 1 + (1 if self.splits else 0)
+    def store_decode(self):
+        """The step as one launch: this step's K/V rows stored inside the decode kernel."""
+        c = self.case
+        self.pa.pa_store_kv_decode(self.k_new, self.v_new, self.slot, self.out, self.q, self.k_cache, self.v_cache,
+                                   self.bt, self.ctx, self.mcl, c.softmax_scale, workspace=self.ws)
 
     def alg_bytes_decode(self):
         c = self.case
@@ -258,33 +263,44 @@ def bench_primary(args, world, rank, device, pk):
     from paged_kv_cache_325_b200 import workloads as W
     case = W.WORKLOADS[PRIMARY](poison=False, keep_contiguous=False)
     b = DecodeBench(case, device)
-    st_replay, _g1 = capture(b.store)
-    dec_replay, _g2 = capture(b.decode)
+    # the step: store + decode in one launch (pa_store_kv_decode); the cache rows it writes are the same
+    # every step, so every step does the same work
+    step_replay, _g0 = capture(b.store_decode)
     timer = Timer(device)
-    timer.run([st_replay, dec_replay], max(args.warmup, 3))
+    timer.run([step_replay], max(args.warmup, 3))
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local_gpu_index(device)) as clk:
-        t_store, t_dec = timer.run([st_replay, dec_replay], args.steps)
+        (t_step,) = timer.run([step_replay], args.steps)
     torch.cuda.synchronize()
     barrier(world)
-    local_total = sum(t_store) + sum(t_dec)
-    value, t_max = aggregate(local_total, args.steps * case.batch, world, device)
-    dec_mean = statistics.mean(t_dec)
-    achieved = b.alg_bytes_decode() / dec_mean / 1e9
+    value, t_max = aggregate(sum(t_step), args.steps * case.batch, world, device)
+    step_mean = statistics.mean(t_step)
+    alg = b.alg_bytes_decode() + b.alg_bytes_store()
+    achieved = alg / step_mean / 1e9
     res = {
         "value": value, "ms_per_step": t_max / args.steps * 1e3,
-        "kv_gbps": case.kv_bytes_read() / dec_mean / 1e9,
-        "kv_hbm_frac_of_measured": case.kv_bytes_read() / dec_mean / 1e9 / pk["hbm_gbs"],
-        "kv_hbm_frac_of_8tbs": case.kv_bytes_read() / dec_mean / 1e9 / 8000.0,
-        "store_us": statistics.mean(t_store) * 1e6, "decode_us": dec_mean * 1e6,
-        "roofline": {"kernel": "decode_split_kernel<128> + decode_combine_kernel", "bound": "hbm",
+        "kv_gbps": case.kv_bytes_read() / step_mean / 1e9,
+        "kv_hbm_frac_of_measured": case.kv_bytes_read() / step_mean / 1e9 / pk["hbm_gbs"],
+        "kv_hbm_frac_of_8tbs": case.kv_bytes_read() / step_mean / 1e9 / 8000.0,
+        "store_decode_us": step_mean * 1e6,
+        "roofline": {"kernel": "decode_split_kernel<128> (store fused)", "bound": "hbm",
                      "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
-                     "traffic": recorded_traffic("decode_qwen3_0.6b"),
-                     "alg_bytes_per_launch": b.alg_bytes_decode()},
-        "gpu_launches": b.launches_per_step() * args.steps,
+                     "traffic": recorded_traffic("store_decode_qwen3_0.6b"), "alg_bytes_per_launch": alg},
+        "gpu_launches": args.steps,
         "clocks": clk.summary(),
     }
+    # the same step as two launches (pa_store_kv, then pa_decode), for comparison; rank 0 at N=1
+    if world == 1:
+        st_replay, _g1 = capture(b.store)
+        dec_replay, _g2 = capture(b.decode)
+        timer.run([st_replay, dec_replay], 5)
+        steps2 = max(10, min(args.steps, 500))
+        t_store, t_dec = timer.run([st_replay, dec_replay], steps2)
+        res["separate_launches"] = {"store_us": statistics.mean(t_store) * 1e6,
+                                    "decode_us": statistics.mean(t_dec) * 1e6,
+                                    "tokens_per_s": case.batch / (statistics.mean(t_store) + statistics.mean(t_dec)),
+                                    "steps": steps2}
     res["e2e"] = bench_e2e(b, args, world, device)
     return case, res
 
@@ -303,8 +319,7 @@ def bench_e2e(b, args, world, device):
     def step():
         for name, t in host.items():
             getattr(b, name).copy_(t, non_blocking=True)
-        b.store()
-        b.decode()
+        b.store_decode()
         out_h.copy_(b.out, non_blocking=True)
 
     timer = Timer(device)
@@ -569,10 +584,10 @@ def main(argv=None):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": PRIMARY_DESC, "parallelism": f"replicas x{world}",
                    "l2": "flushed between timed steps (256 MiB write)",
-                   "timing": "per-step CUDA events around CUDA-graph replays of store and decode"},
+                   "timing": "per-step CUDA events around a CUDA-graph replay of pa_store_kv_decode"},
         "kv_gbps": res["kv_gbps"], "kv_hbm_frac_of_measured": res["kv_hbm_frac_of_measured"],
-        "kv_hbm_frac_of_8tbs": res["kv_hbm_frac_of_8tbs"], "store_us": res["store_us"],
-        "decode_us": res["decode_us"], "roofline": rf, "cpu_baseline": cpu, "e2e": res["e2e"],
+        "kv_hbm_frac_of_8tbs": res["kv_hbm_frac_of_8tbs"], "store_decode_us": res["store_decode_us"],
+        "separate_launches": res.get("separate_launches"), "roofline": rf, "cpu_baseline": cpu, "e2e": res["e2e"],
         "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
     }
     if secondary is not None:

@@ -140,8 +140,10 @@ PA_API size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32
  *   context_lens     [batch] int32, each in [1, max_context_len].
  *   max_context_len  host-side upper bound of context_lens (sizes the split).
  *   workspace        device scratch of at least pa_decode_workspace_size()
- *                    bytes (may be NULL when that size is 0).  Its contents
- *                    need no initialisation and are garbage afterwards.
+ *                    bytes, 256-byte aligned (may be NULL when that size is
+ *                    0).  Its contents need no initialisation and are garbage
+ *                    afterwards.  Two calls whose kernels may overlap on the
+ *                    GPU need two workspaces.
  *
  * The work is split along each context (flash-decoding); per-split partial
  * results in the workspace are merged by a second kernel on the same stream.
@@ -151,6 +153,40 @@ PA_API pa_status pa_decode(void *out, const void *q, const void *k_cache, const 
                     int32_t batch, int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads,
                     int32_t head_dim, int32_t num_blocks, int32_t block_size, float softmax_scale,
                     void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream);
+
+/*
+ * pa_store_kv_decode -- pa_store_kv followed by pa_decode, in one kernel launch
+ * (the decode step of the walkthrough, section seven: store_kvcache of this
+ * step's K/V through slot_mapping, then flash_attn_with_kvcache).  Row s of
+ * k / v is the new token of sequence s (num_tokens == batch), stored at slot
+ * slot_mapping[s]; context_lens[s] counts it, as in pa_decode.  Results are
+ * those of pa_store_kv then pa_decode on the same stream: the cache holds the
+ * new rows afterwards, bit for bit, and out is the decode of the updated cache.
+ *
+ * The new token of sequence s is the one at position context_lens[s] - 1, so
+ * slot_mapping[s] must be either negative (a padding row: nothing is stored and
+ * the decode reads the cache as it is) or that position's slot,
+ * block_table[s][(context_lens[s]-1) / block_size] * block_size
+ * + (context_lens[s]-1) % block_size.  A different slot is still written, but
+ * the decode does not see the new row there; checked mode reports it as
+ * PA_DEVERR_SLOT, as it does a slot >= num_blocks * block_size (not written).
+ * A row of a sequence whose context length is invalid is not stored.
+ *
+ *   k, v          [batch, num_kv_heads, head_dim] bf16, row s at element
+ *                 s * k_row_stride (v_row_stride); the rows must be 16-byte
+ *                 aligned (strides a multiple of 8 elements), otherwise
+ *                 PA_ERR_UNSUPPORTED: use pa_store_kv + pa_decode.
+ *   slot_mapping  [batch] int32, device.
+ *   everything else as pa_decode, with the same workspace size
+ *   (pa_decode_workspace_size).
+ */
+PA_API pa_status pa_store_kv_decode(const void *k, const void *v, int64_t k_row_stride, int64_t v_row_stride,
+                                    const int32_t *slot_mapping, void *out, const void *q, void *k_cache,
+                                    void *v_cache, const int32_t *block_table, int32_t block_table_stride,
+                                    const int32_t *context_lens, int32_t batch, int32_t max_context_len,
+                                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                    int32_t num_blocks, int32_t block_size, float softmax_scale, void *workspace,
+                                    size_t workspace_bytes, int32_t *dev_error, void *stream);
 
 /*
  * pa_decode_split -- pa_decode with the number of context splits chosen by

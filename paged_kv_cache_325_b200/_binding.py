@@ -33,6 +33,7 @@ PA_DEVERR_SEQLENS = 0x8
 PA_DEVERR_TIMEOUT = 0x10
 
 __all__ = ["PagedAttnError", "load_library", "declared_symbols", "pa_store_kv", "pa_decode", "pa_decode_split",
+           "pa_store_kv_decode",
            "pa_decode_workspace_size", "pa_decode_split_workspace_size", "pa_decode_noalloc",
            "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size", "alloc_shared_prefix_workspace", "pa_prefill_varlen",
            "pa_prefill_workspace_size", "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
@@ -57,6 +58,9 @@ _SIGS = {
     "pa_decode_split_workspace_size": (_c_sz, [_c_i32] * 6),
     "pa_decode": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_i32,
                                  _c_i32, _c_i32, _c_i32, _c_f32, _c_p, _c_sz, _c_p, _c_p]),
+    "pa_store_kv_decode": (ctypes.c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i32,
+                                          _c_p, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_f32, _c_p,
+                                          _c_sz, _c_p, _c_p]),
     "pa_decode_split": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_i32,
                                        _c_i32, _c_i32, _c_i32, _c_f32, _c_i32, _c_p, _c_sz, _c_p, _c_p]),
     "pa_decode_shared_prefix_workspace_size": (_c_sz, [_c_i32] * 7),
@@ -226,6 +230,27 @@ def pa_decode(out, q, k_cache, v_cache, block_table, context_lens, max_context_l
         st = lib.pa_decode_split(*common, int(num_splits), _ptr(workspace), ws, _opt_err(dev_error, dev),
                                  _stream(q, stream))
     _check(st)
+
+
+def pa_store_kv_decode(k, v, slot_mapping, out, q, k_cache, v_cache, block_table, context_lens, max_context_len,
+                       softmax_scale, workspace=None, dev_error=None, stream=None):
+    """pa_store_kv of this step's rows (row s = sequence s's new token) and pa_decode, in one launch."""
+    import torch
+    nb, B, Hkv, D, batch, Hq, dev = _decode_args(out, q, k_cache, v_cache, block_table, context_lens)
+    for name, t in (("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, dev, contiguous=False)
+        if t.dim() != 3 or tuple(t.shape) != (batch, Hkv, D) or t.stride(2) != 1 or t.stride(1) != D:
+            raise ValueError(f"{name} must be [batch, num_kv_heads, head_dim] with contiguous rows")
+    _need(slot_mapping, "slot_mapping", torch.int32, dev)
+    if tuple(slot_mapping.shape) != (batch,):
+        raise ValueError("slot_mapping must be [batch]")
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if workspace is not None:
+        _need(workspace, "workspace", None, dev)
+    _check(load_library().pa_store_kv_decode(
+        _ptr(k), _ptr(v), k.stride(0), v.stride(0), _ptr(slot_mapping), _ptr(out), _ptr(q), _ptr(k_cache),
+        _ptr(v_cache), _ptr(block_table), block_table.shape[1], _ptr(context_lens), batch, int(max_context_len), Hq,
+        Hkv, D, nb, B, float(softmax_scale), _ptr(workspace), ws, _opt_err(dev_error, dev), _stream(q, stream)))
 
 
 def pa_decode_split(out, q, k_cache, v_cache, block_table, context_lens, max_context_len, softmax_scale,

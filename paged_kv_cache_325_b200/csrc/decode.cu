@@ -1,4 +1,5 @@
-// Paged GQA decode attention: split-KV flash-decoding plus a combine pass.
+// Paged GQA decode attention: split-KV flash-decoding plus a combine pass,
+// optionally with this step's store_kvcache fused into the split kernel.
 //
 // What it computes (per sequence s, q-head h):
 //     out[s, h] = softmax_j(scale * q[s, h] . K_j) V_j  over the context of s,
@@ -8,9 +9,11 @@
 // flash_attn_with_kvcache call of the nano-vllm walkthrough (section seven).
 //
 // How:
-//  * grid (split, kv_head, sequence); each CTA owns `chunk` consecutive tokens
-//    of one sequence's context for one KV head and ALL G q-heads of its GQA
-//    group, so every K/V byte is read from HBM once per call.
+//  * work items (split, sequence, KV head), numbered split-major and dealt
+//    round-robin to persistent CTAs (2 per SM); an item is `chunk` consecutive
+//    tokens of one sequence's context for one KV head and ALL G q-heads of its
+//    GQA group, so every K/V byte is read from HBM once per call, and a CTA's
+//    items stream through one continuous TMA ring.
 //  * warp 4 is a TMA producer: for each 64-token tile it reads the tile's
 //    physical block ids from block_table and issues 3-D tensor-map loads
 //    (128-byte swizzle) of the K and V rows of this KV head into a 3-stage
@@ -25,6 +28,13 @@
 //  * masked positions (past the end of the context) are selected out: their
 //    score becomes -inf and their V rows are zeroed in registers, so stale or
 //    poisoned cache contents never reach the result (0 * NaN is never formed).
+//  * fused store (pa_store_kv_decode): the consumer warp whose 16-token slice
+//    holds position context_len - 1 of the pair's last split copies the new
+//    token's K/V row of its KV head into a staging row at the start of the
+//    item (cp.async), and, once the tile holding that position has landed,
+//    writes it into the tile in shared memory (in place of the cache row the
+//    TMA brought) and to its cache slot in HBM -- the store_kvcache of the
+//    walkthrough, section seven, done inside the attention launch.
 #include <float.h>
 
 #include <atomic>
@@ -49,7 +59,8 @@ struct DecodeCfg {
     static constexpr int kStageBytes = 2 * kKvBytes;
     static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kBarOff = kRingBytes;                   // 256 bytes of barriers
-    static constexpr int kQOff = kBarOff + 256;                  // 2 slots of the group's G q-head rows
+    static constexpr int kNewOff = kBarOff + 256;                // fused store: the new token's K and V row
+    static constexpr int kQOff = kNewOff + 512;                  // 2 slots of the group's G q-head rows
     // then the merge area: per consumer warp, G rows of D partial sums plus (max, sum)
     static constexpr size_t red_off(int G) { return (size_t)kQOff + 2 * (size_t)G * D * 2; }
     static constexpr size_t smem_bytes(int G) {
@@ -66,6 +77,7 @@ __device__ __forceinline__ void consumer_sync() {
 struct DecItem {
     int valid;          // 0: skip (past the context, or an invalid context length)
     int s, kvh, t_begin, t_end, ntiles, split;
+    int ctx;            // context length
 };
 
 __device__ __forceinline__ DecItem dec_item(const DecodeArgs &a, int i, bool report_bad) {
@@ -82,6 +94,7 @@ __device__ __forceinline__ DecItem dec_item(const DecodeArgs &a, int i, bool rep
         if (report_bad && it.split == 0 && it.kvh == 0) report(a.dev_error, PA_DEVERR_CONTEXT_LEN);
         return it;
     }
+    it.ctx = ctx;
     it.t_begin = a.t_offset + it.split * a.plan.chunk;
     if (it.t_begin >= ctx) return it;            // this split lies past the end of the context
     it.t_end = min(ctx, it.t_begin + a.plan.chunk);
@@ -90,7 +103,9 @@ __device__ __forceinline__ DecItem dec_item(const DecodeArgs &a, int i, bool rep
     return it;
 }
 
-template <int D>
+// kFused: the pa_store_kv_decode variant (store fused in); a separate instantiation, so the plain decode
+// carries none of its registers.
+template <int D, bool kFused>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const DecodeArgs a) {
@@ -200,6 +215,41 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
         const DecItem it = dec_item(a, i, false);
         if (!it.valid) continue;
+        // fused store: this warp owns the new token's row if position ctx - 1 falls in its slice of the
+        // pair's last split; the row is staged now and used when its tile lands
+        int own_t = -1;                       // tile (within the item) holding the new token, or -1
+        bool own_patch = false;               // the slot is the row this decode reads: patch the tile too
+        uint32_t own_r = 0;                   // row of the new token in that tile
+        if (kFused && it.t_end == it.ctx && ((it.ctx - 1 - it.t_begin) % kTile) / 16 == warp) {
+            const int32_t sl = __ldg(a.new_slots + it.s);
+            if (sl >= 0) {
+                const int p = it.ctx - 1;
+                const int32_t blk = __ldg(a.block_table + (int64_t)it.s * a.bt_stride + p / a.block_size);
+                const int64_t expect = (int64_t)blk * a.block_size + p % a.block_size;
+                if ((int64_t)sl >= a.num_slots) {
+                    if (lane == 0) report(a.dev_error, PA_DEVERR_SLOT);
+                } else {
+                    // a slot other than the row this decode reads is still written (as pa_store_kv would)
+                    if (sl != expect && lane == 0) report(a.dev_error, PA_DEVERR_SLOT);
+                    own_t = (p - it.t_begin) / kTile;
+                    own_r = (uint32_t)((p - it.t_begin) % kTile);
+                    own_patch = sl == expect;
+                    // lane c < D/8 copies 16 bytes of K, lane D/8 + c those of V, into the staging row
+                    // (asynchronously: the latency hides behind the item's earlier tiles)
+                    if (lane < D / 4) {
+                        const bool isv = lane >= D / 8;
+                        const int c = isv ? lane - D / 8 : lane;
+                        const __nv_bfloat16 *src =
+                            static_cast<const __nv_bfloat16 *>(isv ? a.v_new : a.k_new) +
+                            (int64_t)it.s * (isv ? a.vn_stride : a.kn_stride) + (int64_t)it.kvh * D + c * 8;
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ring + C::kNewOff + lane * 16),
+                                     "l"(src)
+                                     : "memory");
+                    }
+                    asm volatile("cp.async.commit_group;" ::: "memory");
+                }
+            }
+        }
         // Q fragments; rows past the group are zero
         const int qs = nqi & 1;
         // After a timed-out wait the consumers keep the same control flow (every warp must still reach
@@ -244,6 +294,30 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint32_t kbase = ring + st * C::kStageBytes;
             const uint32_t vbase = kbase + C::kKvBytes;
             const int tok0 = it.t_begin + t * kTile + warp * 16;   // first token of this warp's slice
+            const bool own_tile = kFused && t == own_t;             // warp-uniform
+            if (own_tile) {
+                asm volatile("cp.async.wait_all;" ::: "memory");   // this lane's staged 16 bytes
+                if (lane < D / 4) {
+                    const bool isv = lane >= D / 8;
+                    const uint32_t c = isv ? lane - D / 8 : lane;
+                    uint4 nrow;
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(nrow.x), "=r"(nrow.y), "=r"(nrow.z), "=r"(nrow.w)
+                                 : "r"(ring + C::kNewOff + lane * 16)
+                                 : "memory");
+                    if (own_patch) {
+                        const uint32_t dst =
+                            (isv ? vbase : kbase) + (c >> 3) * kHalfBytes + swz128(own_r, c & 7);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(nrow.x),
+                                     "r"(nrow.y), "r"(nrow.z), "r"(nrow.w)
+                                     : "memory");
+                    }
+                    __nv_bfloat16 *dstg = static_cast<__nv_bfloat16 *>(isv ? a.v_cache : a.k_cache) +
+                                          ((int64_t)__ldg(a.new_slots + it.s) * a.num_kv_heads + it.kvh) * D + c * 8;
+                    *reinterpret_cast<uint4 *>(dstg) = nrow;
+                }
+                __syncwarp();
+            }
 
             // S = Q K^T over this warp's 16 tokens (two n-tiles of 8 tokens)
             float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -326,6 +400,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mma_bf16_16816(o[2 * jp], pa, b0a, b1a);
                 mma_bf16_16816(o[2 * jp + 1], pa, b0b, b1b);
             }
+            // a patched stage is rewritten by a later TMA load: order the generic writes before it
+            if (own_tile && own_patch) fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(empty + st));
         }
@@ -380,7 +456,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-// Merge the per-split partials of one (sequence, q-head) by log-sum-exp.
+// Merge the per-split partials of one (sequence, q-head) by log-sum-exp.  D threads, one per output
+// element.  Every warp reads the log-sum-exps 32 at a time (one per lane) and reduces them with shuffles;
+// the partial rows are then read in unrolled batches, so a merge costs a few L2 round trips, not two per
+// split.
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
     asm volatile("griddepcontrol.wait;" ::: "memory");   // partials of the split kernel are visible
@@ -394,37 +473,51 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
     const int nsplit = (ctx - a.t_offset + a.plan.chunk - 1) / a.plan.chunk;
     const int n = a.part_base + nsplit;
     const int64_t base = ((int64_t)s * a.num_q_heads + h) * a.part_slots;
+    const int d = threadIdx.x, lane = d & 31;
+    const float *lse = a.part_lse + base;
+    const float *po = a.part_o + base * D + d;
     float mt = -INFINITY;
-    for (int i = 0; i < n; ++i) mt = fmaxf(mt, a.part_lse[base + i]);
-    float den = 0.f, num = 0.f;
-    const int d = threadIdx.x;
-    for (int i = 0; i < n; ++i) {
-        const float w = fast_exp2(a.part_lse[base + i] - mt);
-        den += w;
-        num += w * a.part_o[(base + i) * D + d];
+    for (int k0 = 0; k0 < n; k0 += 32) {
+        float l = k0 + lane < n ? lse[k0 + lane] : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l = fmaxf(l, __shfl_xor_sync(0xffffffffu, l, o));
+        mt = fmaxf(mt, l);
     }
-    static_cast<__nv_bfloat16 *>(a.out)[((int64_t)s * a.num_q_heads + h) * D + d] = __float2bfloat16_rn(num / den);
+    float den_lane = 0.f, num = 0.f;
+    for (int k0 = 0; k0 < n; k0 += 32) {
+        const float l = k0 + lane < n ? lse[k0 + lane] : -INFINITY;
+        const float w = l == -INFINITY ? 0.f : fast_exp2(l - mt);
+        den_lane += w;
+        const int m = min(32, n - k0);
+#pragma unroll 8
+        for (int j = 0; j < m; ++j) num += __shfl_sync(0xffffffffu, w, j) * po[(int64_t)(k0 + j) * D];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den_lane += __shfl_xor_sync(0xffffffffu, den_lane, o);
+    static_cast<__nv_bfloat16 *>(a.out)[((int64_t)s * a.num_q_heads + h) * D + d] =
+        __float2bfloat16_rn(num / den_lane);
 }
 
 template <int D>
 cudaError_t launch_decode_d(const DecodeArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                             cudaStream_t stream) {
     using C = DecodeCfg<D>;
-    // attribute and occupancy per (device, G); G <= 16
-    static std::atomic<int> resident[64][17];
+    const bool fused = a.new_slots != nullptr;
+    auto kernel = fused ? decode_split_kernel<D, true> : decode_split_kernel<D, false>;
+    // attribute and occupancy per (device, variant, G); G <= 16
+    static std::atomic<int> resident[64][2][17];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const size_t smem = C::smem_bytes(a.group);
-    int per_sm = resident[dev & 63][a.group].load(std::memory_order_acquire);
+    int per_sm = resident[dev & 63][fused][a.group].load(std::memory_order_acquire);
     if (per_sm == 0) {
-        e = cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)C::smem_bytes(16));
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::smem_bytes(16));
         if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_split_kernel<D>, kThreads, smem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
         if (e != cudaSuccess) return e;
         if (per_sm < 1) per_sm = 1;
-        resident[dev & 63][a.group].store(per_sm, std::memory_order_release);
+        resident[dev & 63][fused][a.group].store(per_sm, std::memory_order_release);
     }
     int sms = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -432,7 +525,7 @@ cudaError_t launch_decode_d(const DecodeArgs &a, const CUtensorMap &tm_k, const 
     const int64_t n_items = (int64_t)a.plan.max_splits * a.batch * a.num_kv_heads;
     const int64_t slots = (int64_t)per_sm * sms;
     const int grid = (int)(n_items < slots ? n_items : slots);
-    decode_split_kernel<D><<<grid, kThreads, smem, stream>>>(tm_k, tm_v, a);
+    kernel<<<grid, kThreads, smem, stream>>>(tm_k, tm_v, a);
     e = cudaGetLastError();
     if (e != cudaSuccess || (a.plan.max_splits == 1 && !a.force_partial)) return e;
 

@@ -171,12 +171,19 @@ size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_
     return pa::decode_workspace_bytes(plan, batch, num_q_heads, head_dim);
 }
 
+// The new token rows of pa_store_kv_decode (NULL for the plain decode).
+struct FusedStore {
+    const void *k, *v;
+    int64_t k_row_stride, v_row_stride;
+    const int32_t *slot_mapping;
+};
+
 static pa_status decode_impl(void *out, const void *q, const void *k_cache, const void *v_cache,
                              const int32_t *block_table, int32_t block_table_stride, const int32_t *context_lens,
                              int32_t batch, int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads,
                              int32_t head_dim, int32_t num_blocks, int32_t block_size, float softmax_scale,
                              int32_t num_splits, void *workspace, size_t workspace_bytes, int32_t *dev_error,
-                             void *stream) {
+                             void *stream, const FusedStore *fs = nullptr) {
     if (batch < 0) return fail(PA_ERR_INVALID_ARG, "batch < 0");
     pa_status st = check_cache_shape(num_blocks, block_size, num_kv_heads, head_dim);
     if (st != PA_OK) return st;
@@ -192,8 +199,19 @@ static pa_status decode_impl(void *out, const void *q, const void *k_cache, cons
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
         !aligned(block_table, 4) || !aligned(context_lens, 4) || (dev_error && !aligned(dev_error, 4)))
         return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
+    if (fs) {
+        const int64_t row = (int64_t)num_kv_heads * head_dim;
+        if (!fs->k || !fs->v || !fs->slot_mapping) return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+        if (fs->k_row_stride < row || fs->v_row_stride < row)
+            return fail(PA_ERR_INVALID_ARG, "row strides must be >= num_kv_heads * head_dim");
+        if (fs->k_row_stride % 8 != 0 || fs->v_row_stride % 8 != 0 || !aligned(fs->k, 16) || !aligned(fs->v, 16))
+            return fail(PA_ERR_UNSUPPORTED,
+                        "the fused store needs 16-byte aligned k/v rows (row strides a multiple of 8 elements); "
+                        "use pa_store_kv then pa_decode");
+        if (!aligned(fs->slot_mapping, 4)) return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
+    }
 
-    pa::DecodeArgs a;
+    pa::DecodeArgs a = {};
     a.plan = pa::plan_decode(batch, num_kv_heads, max_context_len, num_splits, num_sms_current());
     const size_t need = pa::decode_workspace_bytes(a.plan, batch, num_q_heads, head_dim);
     if (need > 0) {
@@ -228,6 +246,14 @@ static pa_status decode_impl(void *out, const void *q, const void *k_cache, cons
     a.t_offset = 0;
     a.force_partial = 0;
     a.shared_blocks = 0;
+    a.k_new = fs ? fs->k : nullptr;
+    a.v_new = fs ? fs->v : nullptr;
+    a.kn_stride = fs ? fs->k_row_stride : 0;
+    a.vn_stride = fs ? fs->v_row_stride : 0;
+    a.new_slots = fs ? fs->slot_mapping : nullptr;
+    a.k_cache = const_cast<void *>(k_cache);
+    a.v_cache = const_cast<void *>(v_cache);
+    a.num_slots = (int64_t)num_blocks * block_size;
 
     CUtensorMap tm_k, tm_v;
     const int64_t rows = (int64_t)num_blocks * block_size;
@@ -246,6 +272,18 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     return decode_impl(out, q, k_cache, v_cache, block_table, block_table_stride, context_lens, batch,
                        max_context_len, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, softmax_scale,
                        0, workspace, workspace_bytes, dev_error, stream);
+}
+
+pa_status pa_store_kv_decode(const void *k, const void *v, int64_t k_row_stride, int64_t v_row_stride,
+                             const int32_t *slot_mapping, void *out, const void *q, void *k_cache, void *v_cache,
+                             const int32_t *block_table, int32_t block_table_stride, const int32_t *context_lens,
+                             int32_t batch, int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads,
+                             int32_t head_dim, int32_t num_blocks, int32_t block_size, float softmax_scale,
+                             void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream) {
+    const FusedStore fs = {k, v, k_row_stride, v_row_stride, slot_mapping};
+    return decode_impl(out, q, k_cache, v_cache, block_table, block_table_stride, context_lens, batch,
+                       max_context_len, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, softmax_scale,
+                       0, workspace, workspace_bytes, dev_error, stream, &fs);
 }
 
 size_t pa_decode_split_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
@@ -401,7 +439,7 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
 
     // 2. private suffixes: split-KV decode from token nprefix on, partials after the prefix chunks;
     // 3. the combine kernel merges all partials of each (sequence, q-head)
-    pa::DecodeArgs da;
+    pa::DecodeArgs da = {};
     da.plan = sp.dplan;
     da.out = out;
     da.q = q;
@@ -426,6 +464,7 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
     da.t_offset = nprefix;
     da.force_partial = 1;
     da.shared_blocks = num_shared_blocks;
+    da.num_slots = rows;
     CUtensorMap dk, dv;
     if ((st = encode_rows(&dk, k_cache, rows, num_kv_heads, head_dim, 1, da.box_tokens)) != PA_OK) return st;
     if ((st = encode_rows(&dv, v_cache, rows, num_kv_heads, head_dim, 1, da.box_tokens)) != PA_OK) return st;

@@ -41,8 +41,8 @@ struct DecodeArgs {
     const int32_t *block_table;
     const int32_t *context_lens;
     int32_t *dev_error;
-    float *part_o;      // [batch, Hq, max_splits, D]
-    float *part_lse;    // [batch, Hq, max_splits]
+    float *part_o;      // [batch, Hq, part_slots, D]
+    float *part_lse;    // [batch, Hq, part_slots]
     int32_t bt_stride, batch, num_q_heads, num_kv_heads, group, head_dim;
     int32_t num_blocks, block_size, box_tokens, max_context_len;
     DecodePlan plan;
@@ -52,6 +52,13 @@ struct DecodeArgs {
     int32_t t_offset;        // the split ranges start at this token (shared-prefix decode: P * block_size)
     int32_t force_partial;   // write partials (and run the combine) even with one split
     int32_t shared_blocks;   // checked mode: block_table[s][0..shared_blocks) must equal row 0's
+    // store fused into the decode (pa_store_kv_decode): row s of k_new / v_new is sequence s's new token,
+    // written to cache slot new_slots[s] (skipped when < 0); NULL new_slots: no store
+    const void *k_new, *v_new;
+    int64_t kn_stride, vn_stride;   // elements, multiples of 8
+    const int32_t *new_slots;
+    void *k_cache, *v_cache;
+    int64_t num_slots;
 };
 cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                           cudaStream_t stream);

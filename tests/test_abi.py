@@ -86,6 +86,28 @@ def test_decode_validation(lib):
     assert _decode(lib, maxc=32768, batch=8, ws=A, wsb=16) == pa.PA_ERR_WORKSPACE
 
 
+def _store_decode(lib, **kw):
+    a = dict(k=A, v=A, ks=1024, vs=1024, slots=A, out=A, q=A, kc=A, vc=A, bt=A, bts=4, ctx=A, batch=2, maxc=1000,
+             Hq=32, Hkv=8, D=128, nb=16, B=256, scale=0.088, ws=None, wsb=0, err=None)
+    a.update(kw)
+    return lib.pa_store_kv_decode(a["k"], a["v"], a["ks"], a["vs"], a["slots"], a["out"], a["q"], a["kc"], a["vc"],
+                                  a["bt"], a["bts"], a["ctx"], a["batch"], a["maxc"], a["Hq"], a["Hkv"], a["D"],
+                                  a["nb"], a["B"], a["scale"], a["ws"], a["wsb"], a["err"], None)
+
+
+def test_store_decode_validation(lib):
+    assert _store_decode(lib, k=None) == pa.PA_ERR_INVALID_ARG
+    assert _store_decode(lib, slots=None) == pa.PA_ERR_INVALID_ARG
+    assert _store_decode(lib, ks=1000) == pa.PA_ERR_INVALID_ARG            # shorter than one row
+    assert _store_decode(lib, ks=1028) == pa.PA_ERR_UNSUPPORTED            # rows not 16-byte aligned
+    assert _store_decode(lib, v=MIS) == pa.PA_ERR_UNSUPPORTED
+    assert "pa_store_kv then pa_decode" in lib.pa_last_error_detail().decode()
+    assert _store_decode(lib, slots=MIS) == pa.PA_ERR_INVALID_ARG
+    assert _store_decode(lib, D=96) == pa.PA_ERR_UNSUPPORTED
+    assert _store_decode(lib, batch=0) == pa.PA_OK
+    assert _store_decode(lib, maxc=32768, batch=8) == pa.PA_ERR_WORKSPACE
+
+
 def test_decode_workspace_size_query():
     assert pa.pa_decode_workspace_size(0, 32, 8, 128, 32768, 256) == 0
     n = pa.pa_decode_workspace_size(8, 32, 8, 128, 32768, 256)

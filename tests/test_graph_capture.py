@@ -5,7 +5,8 @@ walkthrough: CUDA graphs captured at start-up, then replayed) runs here on
 static buffers: a padded batch whose padding rows carry slot_mapping = -1 (the
 store skips them) and a one-token context on a spare block.  Each replay takes
 new inputs copied into the static buffers; the real rows are checked against
-the oracle every step.
+the oracle every step.  Both forms are captured: pa_store_kv then pa_decode,
+and pa_store_kv_decode (the store inside the decode launch).
 """
 import numpy as np
 import pytest
@@ -39,7 +40,8 @@ def _step_case(step, n_real, pad, Hq, Hkv, D, B):
     return case, bt, ctx_all, slots, q, kn, vn
 
 
-def test_store_and_decode_replay_from_a_cuda_graph(cuda_lib):
+@pytest.mark.parametrize("fused", [False, True], ids=["store_then_decode", "pa_store_kv_decode"])
+def test_store_and_decode_replay_from_a_cuda_graph(cuda_lib, fused):
     dev = torch.device("cuda:0")
     n_real, pad, Hq, Hkv, D, B, maxb = 13, 3, 16, 8, 128, 16, 48
     batch = n_real + pad
@@ -58,8 +60,11 @@ def test_store_and_decode_replay_from_a_cuda_graph(cuda_lib):
     ws = pa.alloc_decode_workspace(q, Hkv, max_ctx, B)
 
     def step():
-        pa.pa_store_kv(kn, vn, slots, kc, vc)
-        pa.pa_decode(out, q, kc, vc, bt, ctx, max_ctx, case0.softmax_scale, workspace=ws)
+        if fused:                            # one launch
+            pa.pa_store_kv_decode(kn, vn, slots, out, q, kc, vc, bt, ctx, max_ctx, case0.softmax_scale, workspace=ws)
+        else:
+            pa.pa_store_kv(kn, vn, slots, kc, vc)
+            pa.pa_decode(out, q, kc, vc, bt, ctx, max_ctx, case0.softmax_scale, workspace=ws)
 
     def load(step_no):
         case, bt_h, ctx_h, sl_h, q_h, kn_h, vn_h = _step_case(step_no, n_real, pad, Hq, Hkv, D, B)

@@ -287,7 +287,7 @@ def bench_primary(args, world, rank, device, pk):
         "roofline": {"kernel": "decode_split_kernel<128> (store fused)", "bound": "hbm",
                      "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                      "traffic": recorded_traffic("store_decode_qwen3_0.6b"), "alg_bytes_per_launch": alg},
-        "gpu_launches": args.steps,
+        "gpu_launches": 3 * args.steps,     # per step: planning, decode (store fused in) and combine kernels
         "clocks": clk.summary(),
     }
     # the same step as two launches (pa_store_kv, then pa_decode), for comparison; rank 0 at N=1

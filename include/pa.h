@@ -115,7 +115,8 @@ PA_API pa_status pa_store_kv(const void *k, const void *v, int64_t k_row_stride,
 
 /*
  * Bytes of device workspace pa_decode needs for these sizes on the current
- * device (0 when the decode runs in a single pass with no split).
+ * device (0 only when batch <= 0): the planning kernel's table of work items
+ * and, when a context may be split, the per-split partial results.
  */
 PA_API size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                 int32_t max_context_len, int32_t block_size);
@@ -140,13 +141,15 @@ PA_API size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32
  *   context_lens     [batch] int32, each in [1, max_context_len].
  *   max_context_len  host-side upper bound of context_lens (sizes the split).
  *   workspace        device scratch of at least pa_decode_workspace_size()
- *                    bytes, 256-byte aligned (may be NULL when that size is
- *                    0).  Its contents need no initialisation and are garbage
- *                    afterwards.  Two calls whose kernels may overlap on the
- *                    GPU need two workspaces.
+ *                    bytes, 256-byte aligned.  Its contents need no
+ *                    initialisation and are garbage afterwards.  Two calls
+ *                    whose kernels may overlap on the GPU need two workspaces.
  *
- * The work is split along each context (flash-decoding); per-split partial
- * results in the workspace are merged by a second kernel on the same stream.
+ * Three kernels on `stream`: a one-CTA planning kernel reads context_lens and
+ * writes a longest-first table of work items (a whole (sequence, KV head), or
+ * one split of a context far longer than the average per-CTA load); the
+ * persistent decode kernel takes items from it with an atomic counter; a
+ * combine kernel merges the partial results of split contexts by log-sum-exp.
  */
 PA_API pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
                     const int32_t *block_table, int32_t block_table_stride, const int32_t *context_lens,

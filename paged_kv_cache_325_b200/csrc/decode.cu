@@ -9,12 +9,14 @@
 // flash_attn_with_kvcache call of the nano-vllm walkthrough (section seven).
 //
 // How:
-//  * work items (split, sequence, KV head), numbered split-major and dealt
-//    round-robin to persistent CTAs (2 per SM); an item is `chunk` consecutive
-//    tokens of one sequence's context for one KV head and ALL G q-heads of its
-//    GQA group, so every K/V byte is read from HBM once per call, and a CTA's
-//    items stream through one continuous TMA ring.
-//  * warp 4 is a TMA producer: for each 64-token tile it reads the tile's
+//  * a one-CTA planning kernel writes a longest-first table of work items; an
+//    item is a token range of one sequence's context (all of it, or one split
+//    of a context far longer than the average per-CTA load) for one KV head
+//    and ALL G q-heads of its GQA group, so every K/V byte is read from HBM
+//    once per call.  Persistent CTAs (2 per SM) take items with an atomic
+//    counter and stream them through one continuous TMA ring.
+//  * warp 4 is a TMA producer: it fetches the next item, hands it to the
+//    consumers with the item's Q rows, and for each 64-token tile it reads the tile's
 //    physical block ids from block_table and issues 3-D tensor-map loads
 //    (128-byte swizzle) of the K and V rows of this KV head into a 3-stage
 //    shared-memory ring guarded by mbarriers.
@@ -72,35 +74,154 @@ __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 
-// A work item is (split, sequence, KV head); items are numbered split-major and dealt round-robin to
-// persistent CTAs, so every CTA streams several items through one continuous TMA ring.
-struct DecItem {
-    int valid;          // 0: skip (past the context, or an invalid context length)
-    int s, kvh, t_begin, t_end, ntiles, split;
-    int ctx;            // context length
+// Work items.  The planning kernel (decode_plan_kernel, one CTA, run first) reads the context lengths and
+// writes a table of items (sequence, KV head, split, token range) into the workspace, ordered from the
+// longest to the shortest, plus a hand-out counter.  A pair (sequence, KV head) whose context is at most
+// `whole` tiles is one item; a longer one is cut into splits of `chunk` tiles.  `whole` is the average
+// per-CTA load, so on a mix of lengths (the Qwen3-like workload) nothing is split and no partial is written,
+// and pairs far longer than the average (long context) are cut fine enough to balance.  Persistent CTAs
+// take items from the table with an atomic counter: the longest first, so the short ones fill the tail.
+struct DecPlanHdr {
+    int32_t counter;       // next item to hand out
+    int32_t n_items;
+    int32_t whole;         // tiles: a pair of at most this many tiles is one item (0: always split)
+    int32_t chunk;         // tiles per split of a longer pair
 };
+constexpr int kPlanHdrBytes = 256;
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanBuckets = 1024;          // item lengths (tiles) for the longest-first order; longer share the last
 
-__device__ __forceinline__ DecItem dec_item(const DecodeArgs &a, int i, bool report_bad) {
-    DecItem it;
-    const int per_split = a.batch * a.num_kv_heads;
-    it.split = i / per_split;
-    const int r = i % per_split;
-    it.s = r / a.num_kv_heads;
-    it.kvh = r % a.num_kv_heads;
-    it.valid = 0;
-    const int ctx = __ldg(a.context_lens + it.s);
+// Item: {s, kvh | split << 16, t_begin, t_end}; s < 0 marks the end of the stream in shared memory.
+__device__ __forceinline__ int dec_tiles(const DecodeArgs &a, int s, bool report_bad) {
+    const int ctx = __ldg(a.context_lens + s);
     if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size ||
         ctx < a.t_offset) {
-        if (report_bad && it.split == 0 && it.kvh == 0) report(a.dev_error, PA_DEVERR_CONTEXT_LEN);
-        return it;
+        if (report_bad) report(a.dev_error, PA_DEVERR_CONTEXT_LEN);
+        return 0;
     }
-    it.ctx = ctx;
-    it.t_begin = a.t_offset + it.split * a.plan.chunk;
-    if (it.t_begin >= ctx) return it;            // this split lies past the end of the context
-    it.t_end = min(ctx, it.t_begin + a.plan.chunk);
-    it.ntiles = (it.t_end - it.t_begin + kTile - 1) / kTile;
-    it.valid = 1;
-    return it;
+    return (ctx - a.t_offset + kTile - 1) / kTile;
+}
+
+// Splits of a pair with `tiles` tiles under (whole, chunk); 0 tiles: no item.
+__device__ __forceinline__ int dec_nsplit(int tiles, int whole, int chunk) {
+    if (tiles == 0) return 0;
+    return tiles <= whole ? 1 : (tiles + chunk - 1) / chunk;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeArgs a, int32_t num_ctas) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the decode kernel may start its set-up
+    __shared__ unsigned long long s_total;
+    __shared__ int s_off[kPlanBuckets];
+    const int tid = threadIdx.x;
+    if (tid == 0) s_total = 0;
+    for (int b = tid; b < kPlanBuckets; b += kPlanThreads) s_off[b] = 0;
+    __syncthreads();
+    // total work in tiles; checked mode: context lengths and the shared blocks
+    unsigned long long part = 0;
+    for (int s = tid; s < a.batch; s += kPlanThreads) {
+        part += (unsigned long long)dec_tiles(a, s, true) * a.num_kv_heads;
+        if (a.dev_error && a.shared_blocks > 0)
+            for (int b = 0; b < a.shared_blocks; ++b)
+                if (__ldg(a.block_table + (int64_t)s * a.bt_stride + b) != __ldg(a.block_table + b))
+                    report(a.dev_error, PA_DEVERR_BLOCK_ID);
+    }
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((tid & 31) == 0) atomicAdd(&s_total, part);
+    __syncthreads();
+    // split rule: pairs up to the average per-CTA load stay whole; longer ones are cut into pieces of an
+    // eighth of it (never finer than the host's chunk, which sized the partial slots)
+    int whole, chunk;
+    const int host_chunk = a.plan.chunk / kTile;
+    if (a.plan.fixed) {
+        whole = 0;
+        chunk = host_chunk;
+    } else {
+        const unsigned long long avg = (s_total + num_ctas - 1) / (unsigned long long)num_ctas;
+        whole = (int)min(avg, 1ull << 30);
+        if (whole < 4) whole = 4;
+        chunk = (int)min((avg + 7) / 8, 1ull << 30);
+        if (chunk < host_chunk) chunk = host_chunk;
+    }
+    // longest-first order: count items per length bucket, then exclusive offsets from the longest bucket
+    auto bucket = [](int tiles) { return min(tiles, kPlanBuckets - 1); };
+    for (int s = tid; s < a.batch; s += kPlanThreads) {
+        const int tiles = dec_tiles(a, s, false);
+        const int n = dec_nsplit(tiles, whole, chunk);
+        if (n == 0) continue;
+        if (n == 1) {
+            atomicAdd(&s_off[bucket(tiles)], a.num_kv_heads);
+        } else {
+            atomicAdd(&s_off[bucket(chunk)], (n - 1) * a.num_kv_heads);
+            atomicAdd(&s_off[bucket(tiles - (n - 1) * chunk)], a.num_kv_heads);
+        }
+    }
+    __syncthreads();
+    {   // exclusive scan over the buckets from the longest down: thread t owns bucket kPlanBuckets - 1 - t
+        static_assert(kPlanBuckets == kPlanThreads, "one bucket per thread");
+        __shared__ int s_warp[kPlanThreads / 32];
+        const int b = kPlanBuckets - 1 - tid, lane = tid & 31, w = tid >> 5;
+        const int v = s_off[b];
+        int inc = v;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        if (lane == 31) s_warp[w] = inc;
+        __syncthreads();
+        if (w == 0) {
+            int t = s_warp[lane];
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, t, o);
+                if (lane >= o) t += y;
+            }
+            s_warp[lane] = t;               // inclusive totals of warps 0..lane
+        }
+        __syncthreads();
+        s_off[b] = inc - v + (w > 0 ? s_warp[w - 1] : 0);
+        if (tid == kPlanThreads - 1) {
+            DecPlanHdr *h = reinterpret_cast<DecPlanHdr *>(a.plan_ws);
+            h->counter = 0;
+            h->n_items = s_warp[kPlanThreads / 32 - 1];
+            h->whole = whole;
+            h->chunk = chunk;
+        }
+    }
+    __syncthreads();
+    int4 *items = reinterpret_cast<int4 *>(reinterpret_cast<char *>(a.plan_ws) + kPlanHdrBytes);
+    const int64_t npairs = (int64_t)a.batch * a.num_kv_heads;
+    for (int64_t pr = tid; pr < npairs; pr += kPlanThreads) {
+        const int s = (int)(pr / a.num_kv_heads), kvh = (int)(pr % a.num_kv_heads);
+        const int tiles = dec_tiles(a, s, false);
+        const int n = dec_nsplit(tiles, whole, chunk);
+        if (n == 0) continue;
+        const int ctx = __ldg(a.context_lens + s);
+        if (n == 1) {
+            items[atomicAdd(&s_off[bucket(tiles)], 1)] = make_int4(s, kvh, a.t_offset, ctx);
+            continue;
+        }
+        const int ct = chunk * kTile;
+        int pos = atomicAdd(&s_off[bucket(chunk)], n - 1);
+        for (int j = 0; j < n - 1; ++j)
+            items[pos + j] = make_int4(s, kvh | (j << 16), a.t_offset + j * ct, a.t_offset + (j + 1) * ct);
+        pos = atomicAdd(&s_off[bucket(tiles - (n - 1) * chunk)], 1);
+        items[pos] = make_int4(s, kvh | ((n - 1) << 16), a.t_offset + (n - 1) * ct, ctx);
+    }
+}
+
+struct DecItem {
+    int s, kvh, split, t_begin, t_end, ntiles, ctx;
+};
+
+// A consumer-wide vote (the 128 threads of warps 0-3, named barrier 1): true iff v is true for all.
+__device__ __forceinline__ bool consumers_all(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "n"(kConsumerWarps * 32)
+        : "memory");
+    return r != 0;
 }
 
 // kFused: the pa_store_kv_decode variant (store fused in); a separate instantiation, so the plain decode
@@ -120,8 +241,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     float *red_o = reinterpret_cast<float *>(smem + C::red_off(G));   // [warp][G][D]
     float *red_ml = red_o + kConsumerWarps * G * D;                 // [warp][G][2]
 
+    int4 *desc = reinterpret_cast<int4 *>(smem + C::kBarOff + 192);   // [2]: the item of each Q slot
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_items = a.plan.max_splits * a.batch * a.num_kv_heads;
     const uint32_t ring = smem_u32(smem);
     const uint32_t qsm = ring + C::kQOff;
     const uint32_t qslot = (uint32_t)(G * D * 2);
@@ -141,37 +262,54 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------ producer --
+        // One thread.  The next item's index is taken when three tiles of the current item remain to be
+        // issued (not earlier: an item taken early is held back from idle CTAs) and its record is read a tile
+        // later, so both latencies run under the copies already in the ring.  (Reading each tile's block ids
+        // a tile ahead measured slower than reading them just before the copy.)
         if (lane == 0) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             const int B = a.block_size, box = a.box_tokens;
             uint32_t gt = 0, nqi = 0;             // tiles and Q copies issued so far
             bool ok = true;
-            for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x) {
-                const DecItem it = dec_item(a, i, true);
-                if (!it.valid) continue;
-                // Q rows of the GQA group: one contiguous bulk copy
+            asm volatile("griddepcontrol.wait;" ::: "memory");   // the planning kernel's table is complete
+            DecPlanHdr *hdr = reinterpret_cast<DecPlanHdr *>(a.plan_ws);
+            const int4 *items = reinterpret_cast<const int4 *>(reinterpret_cast<const char *>(a.plan_ws) + kPlanHdrBytes);
+            const int n_items = __ldcg(&hdr->n_items);
+            const int4 kEnd = make_int4(-1, 0, 0, 0);
+            int idx = atomicAdd(&hdr->counter, 1);
+            int4 d = idx < n_items ? __ldcg(items + idx) : kEnd;
+            while (ok) {
                 const int qs = nqi & 1;
                 if (nqi >= 2 && !mbar_wait(smem_u32(qempty + qs), ((nqi >> 1) - 1) & 1, a.dev_error)) break;
+                if (d.x < 0) {                    // end of the stream: an item with s < 0, no copy
+                    desc[qs] = d;
+                    mbar_arrive(smem_u32(qfull + qs));
+                    ++nqi;
+                    break;
+                }
+                int idx_next = n_items;
+                int4 d_next = kEnd;
+                desc[qs] = d;                     // the item rides in the Q slot's descriptor
+                const int s = d.x, kvh = d.y & 0xffff, t_begin = d.z, t_end = d.w;
+                const int ntiles = (t_end - t_begin + kTile - 1) / kTile;
+                // Q rows of the GQA group: one contiguous bulk copy
                 const uint32_t qbytes = (uint32_t)(G * D * 2);
                 mbar_arrive_expect_tx(smem_u32(qfull + qs), qbytes);
                 bulk_load(qsm + qs * qslot,
-                          static_cast<const __nv_bfloat16 *>(a.q) + ((int64_t)it.s * a.num_q_heads + (int64_t)it.kvh * G) * D,
+                          static_cast<const __nv_bfloat16 *>(a.q) + ((int64_t)s * a.num_q_heads + (int64_t)kvh * G) * D,
                           qbytes, smem_u32(qfull + qs));
                 ++nqi;
-                const int32_t *bt = a.block_table + (int64_t)it.s * a.bt_stride;
-                if (a.dev_error && a.shared_blocks > 0 && it.split == 0 && it.kvh == 0)
-                    for (int b = 0; b < a.shared_blocks; ++b)
-                        if (__ldg(bt + b) != __ldg(a.block_table + b)) report(a.dev_error, PA_DEVERR_BLOCK_ID);
-                for (int t = 0; t < it.ntiles; ++t, ++gt) {
+                const int32_t *bt = a.block_table + (int64_t)s * a.bt_stride;
+                for (int t = 0; t < ntiles; ++t, ++gt) {
                     const int st = gt % C::kStages;
                     if (gt >= (uint32_t)C::kStages &&
                         !mbar_wait(smem_u32(empty + st), ((gt / C::kStages) & 1) ^ 1, a.dev_error)) {
                         ok = false;
                         break;
                     }
-                    const int tile0 = it.t_begin + t * kTile;
-                    const int nbox = (min(kTile, it.t_end - tile0) + box - 1) / box;
+                    const int tile0 = t_begin + t * kTile;
+                    const int nbox = (min(kTile, t_end - tile0) + box - 1) / box;
                     const uint32_t fb = smem_u32(full + st);
                     mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * 128 * C::kHalves * 2));
                     const uint32_t kdst = ring + st * C::kStageBytes;
@@ -189,14 +327,19 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                         for (int h = 0; h < C::kHalves; ++h) {
                             const uint32_t off = h * kHalfBytes + b * box * 128;
-                            tma_load_3d(kdst + off, &tm_k, h * 64, it.kvh, row, fb);
-                            tma_load_3d(vdst + off, &tm_v, h * 64, it.kvh, row, fb);
+                            tma_load_3d(kdst + off, &tm_k, h * 64, kvh, row, fb);
+                            tma_load_3d(vdst + off, &tm_v, h * 64, kvh, row, fb);
                         }
                     }
+                    // the next item: index and record, issued now and used when this item's copies are out
+                    if (t == max(0, ntiles - 3)) idx_next = atomicAdd(&hdr->counter, 1);
+                    if (t == max(0, ntiles - 2)) d_next = idx_next < n_items ? __ldcg(items + idx_next) : kEnd;
                 }
+                d = d_next;
             }
-            // leave no copy in flight: wait (bounded) for the last load of every stage and the last Q copies;
-            // on the normal path the consumers have already waited for them all and these return at once
+            // leave no copy in flight: wait (bounded) for the last load of every stage and the last Q copies
+            // (the end marker's slot completes by its plain arrive); on the normal path the consumers have
+            // already waited for them all and these return at once
             for (uint32_t i = (gt > (uint32_t)C::kStages ? gt - C::kStages : 0); i < gt; ++i)
                 mbar_wait(smem_u32(full + i % C::kStages), (i / C::kStages) & 1, a.dev_error);
             for (uint32_t i = (nqi > 2 ? nqi - 2 : 0); i < nqi; ++i)
@@ -209,17 +352,28 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int g0 = lane >> 2;             // accumulator rows g0 and g0 + 8
     const int c2 = (lane & 3) * 2;        // accumulator columns c2, c2 + 1
     const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: matrix index / row this lane addresses
-    const bool single = a.plan.max_splits == 1 && !a.force_partial;
     uint32_t gt = 0, nqi = 0;
     bool ok = true;
-    for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
-        const DecItem it = dec_item(a, i, false);
-        if (!it.valid) continue;
+    for (;;) {
+        // the next item, from the producer; the consumers leave together at the end marker or after a
+        // timed-out wait (a wait that gave up leaves the results garbage and dev_error says so)
+        const int qs = nqi & 1;
+        const bool landed = ok && mbar_wait(smem_u32(qfull + qs), (nqi >> 1) & 1, a.dev_error);
+        const int4 d = desc[qs];
+        if (!consumers_all(landed && d.x >= 0)) break;
+        DecItem it;
+        it.s = d.x;
+        it.kvh = d.y & 0xffff;
+        it.split = d.y >> 16;
+        it.t_begin = d.z;
+        it.t_end = d.w;
+        it.ntiles = (it.t_end - it.t_begin + kTile - 1) / kTile;
+        it.ctx = __ldg(a.context_lens + it.s);
         // fused store: this warp owns the new token's row if position ctx - 1 falls in its slice of the
         // pair's last split; the row is staged now and used when its tile lands
-        int own_t = -1;                       // tile (within the item) holding the new token, or -1
-        bool own_patch = false;               // the slot is the row this decode reads: patch the tile too
-        uint32_t own_r = 0;                   // row of the new token in that tile
+        // own: 0, or 1 (this warp stores the new row) | 2 (the slot is the row this decode reads: the tile is
+        // patched too); the tile and row of the new token follow from ctx - 1 - t_begin
+        int own = 0;
         if (kFused && it.t_end == it.ctx && ((it.ctx - 1 - it.t_begin) % kTile) / 16 == warp) {
             const int32_t sl = __ldg(a.new_slots + it.s);
             if (sl >= 0) {
@@ -231,9 +385,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 } else {
                     // a slot other than the row this decode reads is still written (as pa_store_kv would)
                     if (sl != expect && lane == 0) report(a.dev_error, PA_DEVERR_SLOT);
-                    own_t = (p - it.t_begin) / kTile;
-                    own_r = (uint32_t)((p - it.t_begin) % kTile);
-                    own_patch = sl == expect;
+                    own = sl == expect ? 3 : 1;
                     // lane c < D/8 copies 16 bytes of K, lane D/8 + c those of V, into the staging row
                     // (asynchronously: the latency hides behind the item's earlier tiles)
                     if (lane < D / 4) {
@@ -251,13 +403,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
         // Q fragments; rows past the group are zero
-        const int qs = nqi & 1;
-        // After a timed-out wait the consumers keep the same control flow (every warp must still reach
-        // the merge barriers) but stop waiting; the results are garbage and dev_error says so.
-        {
-            const bool landed = ok && mbar_wait(smem_u32(qfull + qs), (nqi >> 1) & 1, a.dev_error);
-            if (!__all_sync(0xffffffffu, landed)) ok = false;
-        }
         ++nqi;
         uint32_t qa[D / 16][4];
         {
@@ -294,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint32_t kbase = ring + st * C::kStageBytes;
             const uint32_t vbase = kbase + C::kKvBytes;
             const int tok0 = it.t_begin + t * kTile + warp * 16;   // first token of this warp's slice
-            const bool own_tile = kFused && t == own_t;             // warp-uniform
+            const bool own_tile = kFused && own != 0 && t == (it.ctx - 1 - it.t_begin) / kTile;   // warp-uniform
             if (own_tile) {
                 asm volatile("cp.async.wait_all;" ::: "memory");   // this lane's staged 16 bytes
                 if (lane < D / 4) {
@@ -305,9 +450,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                                  : "=r"(nrow.x), "=r"(nrow.y), "=r"(nrow.z), "=r"(nrow.w)
                                  : "r"(ring + C::kNewOff + lane * 16)
                                  : "memory");
-                    if (own_patch) {
+                    if (own & 2) {
                         const uint32_t dst =
-                            (isv ? vbase : kbase) + (c >> 3) * kHalfBytes + swz128(own_r, c & 7);
+                            (isv ? vbase : kbase) + (c >> 3) * kHalfBytes + swz128((uint32_t)((it.ctx - 1 - it.t_begin) % kTile), c & 7);
                         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(nrow.x),
                                      "r"(nrow.y), "r"(nrow.z), "r"(nrow.w)
                                      : "memory");
@@ -401,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mma_bf16_16816(o[2 * jp + 1], pa, b0b, b1b);
             }
             // a patched stage is rewritten by a later TMA load: order the generic writes before it
-            if (own_tile && own_patch) fence_proxy_async_smem();
+            if (own_tile && (own & 2)) fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(empty + st));
         }
@@ -429,6 +574,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
         consumer_sync();
+        // the pair's only item and nothing merged in from elsewhere: write the result directly
+        const bool direct = a.part_base == 0 && it.t_begin == a.t_offset && it.t_end == it.ctx;
         for (int e = threadIdx.x; e < G * D; e += kConsumerWarps * 32) {
             const int g = e / D, d = e % D;
             float mt = -INFINITY;
@@ -443,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 ot += f * red_o[(w * G + g) * D + d];
             }
             const int h = it.kvh * G + g;
-            if (single) {
+            if (direct) {
                 static_cast<__nv_bfloat16 *>(a.out)[((int64_t)it.s * a.num_q_heads + h) * D + d] =
                     __float2bfloat16_rn(ot / lt);
             } else {
@@ -469,8 +616,11 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
     if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size ||
         ctx < a.t_offset)
         return;
-    // partials: part_base slots written before this launch (shared-prefix chunks), then the splits
-    const int nsplit = (ctx - a.t_offset + a.plan.chunk - 1) / a.plan.chunk;
+    // partials: part_base slots written before this launch (shared-prefix chunks), then the splits, cut as
+    // the planning kernel cut them; a pair of one split and nothing else was written directly
+    const DecPlanHdr *hdr = reinterpret_cast<const DecPlanHdr *>(a.plan_ws);
+    const int nsplit = dec_nsplit((ctx - a.t_offset + kTile - 1) / kTile, __ldcg(&hdr->whole), __ldcg(&hdr->chunk));
+    if (a.part_base == 0 && nsplit <= 1) return;
     const int n = a.part_base + nsplit;
     const int64_t base = ((int64_t)s * a.num_q_heads + h) * a.part_slots;
     const int d = threadIdx.x, lane = d & 31;
@@ -522,23 +672,32 @@ cudaError_t launch_decode_d(const DecodeArgs &a, const CUtensorMap &tm_k, const 
     int sms = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    const int64_t n_items = (int64_t)a.plan.max_splits * a.batch * a.num_kv_heads;
+    const int64_t n_items = (int64_t)a.plan.max_splits * a.batch * a.num_kv_heads;   // an upper bound
     const int64_t slots = (int64_t)per_sm * sms;
     const int grid = (int)(n_items < slots ? n_items : slots);
-    kernel<<<grid, kThreads, smem, stream>>>(tm_k, tm_v, a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess || (a.plan.max_splits == 1 && !a.force_partial)) return e;
 
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(a.batch * a.num_q_heads));
-    cfg.blockDim = dim3(D);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
+    // 1. the item table; 2. the persistent decode, launched as its programmatic dependent so that its
+    // set-up overlaps the planning (its producer waits for the table with griddepcontrol.wait);
+    // 3. the combine, for pairs that were split
+    decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(a, grid);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, tm_k, tm_v, a);
+    if (e != cudaSuccess || (a.plan.max_splits == 1 && a.part_base == 0)) return e;
+
+    cfg.gridDim = dim3((unsigned)(a.batch * a.num_q_heads));
+    cfg.blockDim = dim3(D);
+    cfg.dynamicSmemBytes = 0;
     return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, a);
 }
 
@@ -566,15 +725,26 @@ DecodePlan plan_decode(int32_t batch, int32_t num_kv_heads, int32_t max_context_
     p.chunk = (int32_t)chunk;
     p.max_splits = (int32_t)((max_context_len + chunk - 1) / chunk);
     if (p.max_splits < 1) p.max_splits = 1;
+    p.fixed = num_splits > 0;
     return p;
 }
 
-size_t decode_workspace_bytes(const DecodePlan &plan, int32_t batch, int32_t num_q_heads, int32_t head_dim,
-                              int32_t extra_slots) {
-    if (plan.max_splits <= 1 && extra_slots == 0) return 0;
+size_t decode_plan_bytes(const DecodePlan &plan, int32_t batch, int32_t num_kv_heads) {
+    const size_t items = (size_t)batch * num_kv_heads * (plan.max_splits > 0 ? plan.max_splits : 1);
+    return (kPlanHdrBytes + items * sizeof(int4) + 255) / 256 * 256;
+}
+
+DecodeWorkspace decode_workspace_layout(const DecodePlan &plan, int32_t batch, int32_t num_q_heads,
+                                        int32_t num_kv_heads, int32_t head_dim, int32_t extra_slots) {
+    auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
+    DecodeWorkspace w;
+    w.plan_off = 0;
+    w.o_off = w.lse_off = w.total = decode_plan_bytes(plan, batch, num_kv_heads);
+    if (plan.max_splits <= 1 && extra_slots == 0) return w;
     const size_t n = (size_t)batch * num_q_heads * (plan.max_splits + extra_slots);
-    const size_t o_bytes = (n * head_dim * sizeof(float) + 255) / 256 * 256;
-    return o_bytes + n * sizeof(float);
+    w.lse_off = w.o_off + r256(n * head_dim * sizeof(float));
+    w.total = w.lse_off + r256(n * sizeof(float));
+    return w;
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,

@@ -168,7 +168,7 @@ size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_
     (void)block_size;
     if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
     pa::DecodePlan plan = pa::plan_decode(batch, num_kv_heads, max_context_len, 0, num_sms_current());
-    return pa::decode_workspace_bytes(plan, batch, num_q_heads, head_dim);
+    return pa::decode_workspace_layout(plan, batch, num_q_heads, num_kv_heads, head_dim).total;
 }
 
 // The new token rows of pa_store_kv_decode (NULL for the plain decode).
@@ -213,23 +213,24 @@ static pa_status decode_impl(void *out, const void *q, const void *k_cache, cons
 
     pa::DecodeArgs a = {};
     a.plan = pa::plan_decode(batch, num_kv_heads, max_context_len, num_splits, num_sms_current());
-    const size_t need = pa::decode_workspace_bytes(a.plan, batch, num_q_heads, head_dim);
-    if (need > 0) {
-        if (!workspace || workspace_bytes < need)
-            return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
-                        workspace ? workspace_bytes : (size_t)0);
-        if (!aligned(workspace, 256)) return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-    }
+    if (a.plan.max_splits > pa::kDecodeMaxSplits || num_kv_heads > pa::kDecodeMaxKvHeads)
+        return fail(PA_ERR_UNSUPPORTED, "more than %d context splits or %d KV heads", pa::kDecodeMaxSplits,
+                    pa::kDecodeMaxKvHeads);
+    const pa::DecodeWorkspace wl = pa::decode_workspace_layout(a.plan, batch, num_q_heads, num_kv_heads, head_dim);
+    const size_t need = wl.total;
+    if (!workspace || workspace_bytes < need)
+        return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (!aligned(workspace, 256)) return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     a.out = out;
     a.q = q;
     a.block_table = block_table;
     a.context_lens = context_lens;
     a.dev_error = dev_error;
-    const size_t n = (size_t)batch * num_q_heads * a.plan.max_splits;
-    a.part_o = static_cast<float *>(workspace);
-    a.part_lse = need ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                                  (n * head_dim * sizeof(float) + 255) / 256 * 256)
-                      : nullptr;
+    char *ws = static_cast<char *>(workspace);
+    a.plan_ws = ws + wl.plan_off;
+    a.part_o = reinterpret_cast<float *>(ws + wl.o_off);
+    a.part_lse = reinterpret_cast<float *>(ws + wl.lse_off);
     a.bt_stride = block_table_stride;
     a.batch = batch;
     a.num_q_heads = num_q_heads;
@@ -244,7 +245,6 @@ static pa_status decode_impl(void *out, const void *q, const void *k_cache, cons
     a.part_slots = a.plan.max_splits;
     a.part_base = 0;
     a.t_offset = 0;
-    a.force_partial = 0;
     a.shared_blocks = 0;
     a.k_new = fs ? fs->k : nullptr;
     a.v_new = fs ? fs->v : nullptr;
@@ -292,7 +292,7 @@ size_t pa_decode_split_workspace_size(int32_t batch, int32_t num_q_heads, int32_
         num_splits < 0)
         return 0;
     pa::DecodePlan plan = pa::plan_decode(batch, num_kv_heads, max_context_len, num_splits, num_sms_current());
-    return pa::decode_workspace_bytes(plan, batch, num_q_heads, head_dim);
+    return pa::decode_workspace_layout(plan, batch, num_q_heads, num_kv_heads, head_dim).total;
 }
 
 pa_status pa_decode_split(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -315,7 +315,7 @@ namespace {
 struct SharedPlan {
     pa::DecodePlan dplan;
     int32_t nchunks, key_chunk, ranks, slots;
-    size_t plan_bytes, o_bytes, lse_bytes, total;
+    size_t plan_bytes, o_bytes, lse_bytes, dplan_bytes, total;
 };
 
 SharedPlan plan_shared(int32_t batch, int32_t Hq, int32_t Hkv, int32_t D, int32_t max_ctx, int32_t B, int32_t P,
@@ -340,7 +340,9 @@ SharedPlan plan_shared(int32_t batch, int32_t Hq, int32_t Hkv, int32_t D, int32_
     sp.plan_bytes = r256(pa::prefill_workspace_bytes(1, batch, G, Hkv, sp.nchunks));
     sp.o_bytes = r256((size_t)batch * Hq * sp.slots * D * sizeof(float));
     sp.lse_bytes = r256((size_t)batch * Hq * sp.slots * sizeof(float));
-    sp.total = sp.plan_bytes + sp.o_bytes + sp.lse_bytes;
+    // the suffix decode's item table (its partials are the slots after the prefix chunks, above)
+    sp.dplan_bytes = pa::decode_plan_bytes(sp.dplan, batch, Hkv);
+    sp.total = sp.plan_bytes + sp.o_bytes + sp.lse_bytes + sp.dplan_bytes;
     return sp;
 }
 
@@ -439,6 +441,9 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
 
     // 2. private suffixes: split-KV decode from token nprefix on, partials after the prefix chunks;
     // 3. the combine kernel merges all partials of each (sequence, q-head)
+    if (sp.dplan.max_splits > pa::kDecodeMaxSplits || num_kv_heads > pa::kDecodeMaxKvHeads)
+        return fail(PA_ERR_UNSUPPORTED, "more than %d context splits or %d KV heads", pa::kDecodeMaxSplits,
+                    pa::kDecodeMaxKvHeads);
     pa::DecodeArgs da = {};
     da.plan = sp.dplan;
     da.out = out;
@@ -448,6 +453,7 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
     da.dev_error = dev_error;
     da.part_o = part_o;
     da.part_lse = part_lse;
+    da.plan_ws = ws + sp.plan_bytes + sp.o_bytes + sp.lse_bytes;
     da.bt_stride = block_table_stride;
     da.batch = batch;
     da.num_q_heads = num_q_heads;
@@ -462,7 +468,6 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
     da.part_slots = sp.slots;
     da.part_base = sp.nchunks;
     da.t_offset = nprefix;
-    da.force_partial = 1;
     da.shared_blocks = num_shared_blocks;
     da.num_slots = rows;
     CUtensorMap dk, dv;

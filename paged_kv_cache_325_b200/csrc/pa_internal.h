@@ -27,13 +27,23 @@ cudaError_t launch_store(const StoreArgs &a, cudaStream_t stream);
 constexpr int kDecodeTileTokens = 64;
 
 struct DecodePlan {
-    int32_t chunk;       // tokens per split, a multiple of kDecodeTileTokens
-    int32_t max_splits;  // splits of the longest context
+    int32_t chunk;       // tokens per split, a multiple of kDecodeTileTokens: the finest split the
+                         // planning kernel may choose (exactly this one when fixed)
+    int32_t max_splits;  // splits of the longest context at that chunk: the partial slots per (s, h)
+    int32_t fixed;       // the caller chose the split count: every pair is cut into chunks of `chunk`
 };
 DecodePlan plan_decode(int32_t batch, int32_t num_kv_heads, int32_t max_context_len, int32_t num_splits,
                        int32_t num_sms);
-size_t decode_workspace_bytes(const DecodePlan &plan, int32_t batch, int32_t num_q_heads, int32_t head_dim,
-                              int32_t extra_slots = 0);
+// Workspace of a decode call: the planning kernel's item table, then (when a pair can be split, or
+// extra_slots partials come from elsewhere) fp32 partials and their log-sum-exps.
+struct DecodeWorkspace {
+    size_t plan_off, o_off, lse_off, total;   // byte offsets from a 256-byte aligned base
+};
+size_t decode_plan_bytes(const DecodePlan &plan, int32_t batch, int32_t num_kv_heads);   // multiple of 256
+DecodeWorkspace decode_workspace_layout(const DecodePlan &plan, int32_t batch, int32_t num_q_heads,
+                                        int32_t num_kv_heads, int32_t head_dim, int32_t extra_slots = 0);
+constexpr int32_t kDecodeMaxSplits = 32767;     // split index and KV head share one int of an item
+constexpr int32_t kDecodeMaxKvHeads = 65535;
 
 struct DecodeArgs {
     void *out;
@@ -41,6 +51,7 @@ struct DecodeArgs {
     const int32_t *block_table;
     const int32_t *context_lens;
     int32_t *dev_error;
+    void *plan_ws;      // the item table (decode_workspace_layout().plan_off)
     float *part_o;      // [batch, Hq, part_slots, D]
     float *part_lse;    // [batch, Hq, part_slots]
     int32_t bt_stride, batch, num_q_heads, num_kv_heads, group, head_dim;
@@ -50,7 +61,6 @@ struct DecodeArgs {
     // the partials of (sequence s, q-head h) sit at slots [part_base, part_base + splits) of part_slots
     int32_t part_slots, part_base;
     int32_t t_offset;        // the split ranges start at this token (shared-prefix decode: P * block_size)
-    int32_t force_partial;   // write partials (and run the combine) even with one split
     int32_t shared_blocks;   // checked mode: block_table[s][0..shared_blocks) must equal row 0's
     // store fused into the decode (pa_store_kv_decode): row s of k_new / v_new is sequence s's new token,
     // written to cache slot new_slots[s] (skipped when < 0); NULL new_slots: no store

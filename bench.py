@@ -402,16 +402,25 @@ def bench_secondary(args, device, pk, names):
         pa.pa_prefill_varlen(o, q, kc, vc, cq, ck, case.max_seqlen_q, case.max_seqlen_k, bt, case.softmax_scale,
                              workspace=pws)
 
+    def fused():
+        pa.pa_store_kv_prefill_varlen(kn, vn, slot, o, q, kc, vc, cq, ck, case.max_seqlen_q, case.max_seqlen_k, bt,
+                                      case.softmax_scale, workspace=pws)
+
     st_replay, _g1 = capture(st)
     pf_replay, _g2 = capture(pf)
+    fu_replay, _g3 = capture(fused)
     timer.run([st_replay, pf_replay], 5)
     ts, tp = timer.run([st_replay, pf_replay], steps)
     tpm, tsm = statistics.mean(tp), statistics.mean(ts)
+    timer.run([fu_replay], 5)
+    (tf,) = timer.run([fu_replay], steps)
+    tfm = statistics.mean(tf)
     fl = case.causal_flops()
     ach = fl / tpm / 1e12
     store_bytes = 2 * 2 * kn.numel() * 2
     out["varlen_prefill"] = {
         "prefill_us": tpm * 1e6, "store_us": tsm * 1e6, "causal_tflop": fl / 1e12,
+        "store_prefill_fused_us": tfm * 1e6, "store_prefill_fused_tflops": fl / tfm / 1e12,
         "tflops": ach, "new_tokens": case.total_q, "prefill_tokens_per_s": case.total_q / (tpm + tsm),
         "store_gbps": store_bytes / tsm / 1e9,
         "roofline": {"kernel": "prefill_kernel<128>", "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],

@@ -315,6 +315,38 @@ PA_API pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, co
                             void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream);
 
 /*
+ * pa_store_kv_prefill_varlen -- pa_store_kv of the prompts' new K/V rows
+ * followed by pa_prefill_varlen, in one launch, with the new keys read
+ * straight from the new K/V rows instead of back from the cache (the prefill
+ * step of the walkthrough, section seven: store_kvcache through slot_mapping,
+ * then flash_attn_varlen_func over the paged cache).  Row cu_seqlens_q[s] + i
+ * of k / v (and of slot_mapping) is sequence s's new token at position c + i,
+ * c = n_k - n_new the cached prefix (whole blocks).  Results are those of
+ * pa_store_kv then pa_prefill_varlen on the same stream: the cache holds the
+ * new rows afterwards, bit for bit, and out is the prefill of the updated
+ * cache -- provided each slot_mapping row is the slot that block_table gives
+ * for that token's position, which checked mode verifies (PA_DEVERR_SLOT; a
+ * negative slot is also reported, and not stored, while the prefill still uses
+ * the row).  No other kernel of the launch reads the stored slots.
+ *
+ *   k, v          [total_q, num_kv_heads, head_dim] bf16, row t at element
+ *                 t * k_row_stride (v_row_stride); 16-byte aligned rows
+ *                 (strides a multiple of 8 elements), otherwise
+ *                 PA_ERR_UNSUPPORTED: use pa_store_kv + pa_prefill_varlen.
+ *   slot_mapping  [total_q] int32, device.
+ *   everything else as pa_prefill_varlen (same workspace size).
+ */
+PA_API pa_status pa_store_kv_prefill_varlen(const void *k, const void *v, int64_t k_row_stride, int64_t v_row_stride,
+                                            const int32_t *slot_mapping, void *out, const void *q, int32_t total_q,
+                                            void *k_cache, void *v_cache, const int32_t *cu_seqlens_q,
+                                            const int32_t *cu_seqlens_k, int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                            const int32_t *block_table, int32_t block_table_stride, int32_t batch,
+                                            int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                            int32_t num_blocks, int32_t block_size, float softmax_scale,
+                                            int32_t causal, void *workspace, size_t workspace_bytes,
+                                            int32_t *dev_error, void *stream);
+
+/*
  * pa_selftest_bounded_wait -- exercises the library's bounded mbarrier wait:
  * one CTA waits for an arrival that never comes, gives up after
  * `max_polls` polls, ORs PA_DEVERR_TIMEOUT into *dev_error and exits

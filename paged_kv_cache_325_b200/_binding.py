@@ -33,7 +33,7 @@ PA_DEVERR_SEQLENS = 0x8
 PA_DEVERR_TIMEOUT = 0x10
 
 __all__ = ["PagedAttnError", "load_library", "declared_symbols", "pa_store_kv", "pa_decode", "pa_decode_split",
-           "pa_store_kv_decode",
+           "pa_store_kv_decode", "pa_store_kv_prefill_varlen",
            "pa_decode_workspace_size", "pa_decode_split_workspace_size", "pa_decode_noalloc",
            "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size", "alloc_shared_prefix_workspace", "pa_prefill_varlen",
            "pa_prefill_workspace_size", "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
@@ -74,6 +74,9 @@ _SIGS = {
     "pa_prefill_varlen": (ctypes.c_int, [_c_p, _c_p, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_i32, _c_p, _c_i32, _c_i32,
                                          _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_f32, _c_i32, _c_p, _c_sz, _c_p,
                                          _c_p]),
+    "pa_store_kv_prefill_varlen": (ctypes.c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_p,
+                                                  _c_p, _c_p, _c_i32, _c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_i32,
+                                                  _c_i32, _c_i32, _c_i32, _c_f32, _c_i32, _c_p, _c_sz, _c_p, _c_p]),
     "pa_selftest_bounded_wait": (ctypes.c_int, [_c_p, _c_i64, _c_p]),
 }
 
@@ -331,6 +334,39 @@ def pa_prefill_varlen(out, q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_
         int(max_seqlen_q), int(max_seqlen_k), _ptr(block_table), block_table.shape[1], batch, q.shape[1], Hkv, D,
         nb, B, float(softmax_scale), int(bool(causal)), _ptr(workspace), ws, _opt_err(dev_error, dev),
         _stream(q, stream)))
+
+
+def pa_store_kv_prefill_varlen(k, v, slot_mapping, out, q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k,
+                               max_seqlen_q, max_seqlen_k, block_table, softmax_scale, causal=True, workspace=None,
+                               dev_error=None, stream=None):
+    """pa_store_kv of the prompts' new rows and pa_prefill_varlen in one launch, the new keys read from k / v."""
+    import torch
+    nb, B, Hkv, D = _cache_dims(k_cache, v_cache)
+    dev = k_cache.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(out, "out", torch.bfloat16, dev)
+    if q.dim() != 3 or q.shape[2] != D or out.shape != q.shape:
+        raise ValueError("q and out must be [total_q, num_q_heads, head_dim]")
+    total_q = int(q.shape[0])
+    for name, t in (("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, dev, contiguous=False)
+        if t.dim() != 3 or tuple(t.shape) != (total_q, Hkv, D) or t.stride(2) != 1 or t.stride(1) != D:
+            raise ValueError(f"{name} must be [total_q, num_kv_heads, head_dim] with contiguous rows")
+    _need(slot_mapping, "slot_mapping", torch.int32, dev)
+    if tuple(slot_mapping.shape) != (total_q,):
+        raise ValueError("slot_mapping must be [total_q]")
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, dev)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, dev)
+    _need(block_table, "block_table", torch.int32, dev)
+    batch = int(cu_seqlens_q.shape[0]) - 1
+    if cu_seqlens_k.shape != cu_seqlens_q.shape or block_table.dim() != 2 or block_table.shape[0] != batch:
+        raise ValueError("cu_seqlens_q/k must be [batch+1] and block_table [batch, max_blocks]")
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().pa_store_kv_prefill_varlen(
+        _ptr(k), _ptr(v), k.stride(0), v.stride(0), _ptr(slot_mapping), _ptr(out), _ptr(q), total_q, _ptr(k_cache),
+        _ptr(v_cache), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q), int(max_seqlen_k),
+        _ptr(block_table), block_table.shape[1], batch, q.shape[1], Hkv, D, nb, B, float(softmax_scale),
+        int(bool(causal)), _ptr(workspace), ws, _opt_err(dev_error, dev), _stream(q, stream)))
 
 
 def pa_selftest_bounded_wait(dev_error, max_polls, stream=None):

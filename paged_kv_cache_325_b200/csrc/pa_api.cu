@@ -72,11 +72,13 @@ int num_sms_current() {
 // first) {head_dim, heads, rows}, box {64, box_heads, box_rows}, 128-byte
 // swizzle (each box row of 64 bf16 values is one 128-byte swizzle row).
 pa_status encode_rows(CUtensorMap *map, const void *base, int64_t rows, int32_t heads, int32_t head_dim,
-                      int32_t box_heads, int32_t box_rows) {
+                      int32_t box_heads, int32_t box_rows, int64_t row_stride = 0) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (no CUDA driver?)");
     cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)heads, (cuuint64_t)rows};
-    cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)heads * head_dim * 2};
+    // row_stride (elements; 0: heads * head_dim) must be a multiple of 8 (the 16-byte stride rule)
+    const int64_t rs = row_stride > 0 ? row_stride : (int64_t)heads * head_dim;
+    cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)rs * 2};
     cuuint32_t box[3] = {64u, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
     cuuint32_t estr[3] = {1u, 1u, 1u};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
@@ -487,12 +489,13 @@ size_t pa_prefill_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t nu
     return pa::prefill_workspace_bytes(batch, max_seqlen_q, num_q_heads / num_kv_heads, num_kv_heads);
 }
 
-pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const void *k_cache, const void *v_cache,
-                            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t max_seqlen_q,
-                            int32_t max_seqlen_k, const int32_t *block_table, int32_t block_table_stride,
-                            int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                            int32_t num_blocks, int32_t block_size, float softmax_scale, int32_t causal,
-                            void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream) {
+static pa_status prefill_impl(void *out, const void *q, int32_t total_q, const void *k_cache, const void *v_cache,
+                              const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t max_seqlen_q,
+                              int32_t max_seqlen_k, const int32_t *block_table, int32_t block_table_stride,
+                              int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                              int32_t num_blocks, int32_t block_size, float softmax_scale, int32_t causal,
+                              void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream,
+                              const FusedStore *fs) {
     if (batch < 0) return fail(PA_ERR_INVALID_ARG, "batch < 0");
     pa_status st = check_cache_shape(num_blocks, block_size, num_kv_heads, head_dim);
     if (st != PA_OK) return st;
@@ -520,8 +523,19 @@ pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const voi
         !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) || !aligned(block_table, 4) ||
         (dev_error && !aligned(dev_error, 4)))
         return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
+    if (fs) {
+        const int64_t row = (int64_t)num_kv_heads * head_dim;
+        if (!fs->k || !fs->v || !fs->slot_mapping) return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+        if (fs->k_row_stride < row || fs->v_row_stride < row)
+            return fail(PA_ERR_INVALID_ARG, "row strides must be >= num_kv_heads * head_dim");
+        if (fs->k_row_stride % 8 != 0 || fs->v_row_stride % 8 != 0 || !aligned(fs->k, 16) || !aligned(fs->v, 16))
+            return fail(PA_ERR_UNSUPPORTED,
+                        "the fused store needs 16-byte aligned k/v rows (row strides a multiple of 8 elements); "
+                        "use pa_store_kv then pa_prefill_varlen");
+        if (!aligned(fs->slot_mapping, 4)) return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
+    }
 
-    pa::PrefillArgs a;
+    pa::PrefillArgs a = {};
     a.out = out;
     a.q = q;
     a.cu_q = cu_seqlens_q;
@@ -557,10 +571,54 @@ pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const voi
     // q viewed as [total_q, Hq, D]: one box is the (128 / G) tokens x G q-heads of one Q tile
     CUtensorMap tm_q;
     if ((st = encode_rows(&tm_q, q, total_q, num_q_heads, head_dim, a.group, 128 / a.group)) != PA_OK) return st;
-    cudaError_t e = pa::launch_prefill(a, tm_q, tm_k, tm_v, static_cast<cudaStream_t>(stream));
+    CUtensorMap tm_kn, tm_vn;
+    if (fs) {
+        a.k_new = fs->k;
+        a.v_new = fs->v;
+        a.kn_stride = fs->k_row_stride;
+        a.vn_stride = fs->v_row_stride;
+        a.new_slots = fs->slot_mapping;
+        a.k_cache = const_cast<void *>(k_cache);
+        a.v_cache = const_cast<void *>(v_cache);
+        a.num_slots = rows;
+        // the new K/V rows as [total_q, Hkv, D] with their row strides, boxes as the cache's
+        if ((st = encode_rows(&tm_kn, fs->k, total_q, num_kv_heads, head_dim, 1, a.box_tokens, fs->k_row_stride)) !=
+            PA_OK)
+            return st;
+        if ((st = encode_rows(&tm_vn, fs->v, total_q, num_kv_heads, head_dim, 1, a.box_tokens, fs->v_row_stride)) !=
+            PA_OK)
+            return st;
+    }
+    cudaError_t e = pa::launch_prefill(a, tm_q, tm_k, tm_v, static_cast<cudaStream_t>(stream), fs ? &tm_kn : nullptr,
+                                       fs ? &tm_vn : nullptr);
     if (e == cudaErrorNotSupported) return fail(PA_ERR_UNSUPPORTED, "prefill kernel not available");
     if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
     return ok();
+}
+
+pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const void *k_cache, const void *v_cache,
+                            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t max_seqlen_q,
+                            int32_t max_seqlen_k, const int32_t *block_table, int32_t block_table_stride,
+                            int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                            int32_t num_blocks, int32_t block_size, float softmax_scale, int32_t causal,
+                            void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream) {
+    return prefill_impl(out, q, total_q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                        block_table, block_table_stride, batch, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                        block_size, softmax_scale, causal, workspace, workspace_bytes, dev_error, stream, nullptr);
+}
+
+pa_status pa_store_kv_prefill_varlen(const void *k, const void *v, int64_t k_row_stride, int64_t v_row_stride,
+                                     const int32_t *slot_mapping, void *out, const void *q, int32_t total_q,
+                                     void *k_cache, void *v_cache, const int32_t *cu_seqlens_q,
+                                     const int32_t *cu_seqlens_k, int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                     const int32_t *block_table, int32_t block_table_stride, int32_t batch,
+                                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t num_blocks,
+                                     int32_t block_size, float softmax_scale, int32_t causal, void *workspace,
+                                     size_t workspace_bytes, int32_t *dev_error, void *stream) {
+    const FusedStore fs = {k, v, k_row_stride, v_row_stride, slot_mapping};
+    return prefill_impl(out, q, total_q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                        block_table, block_table_stride, batch, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                        block_size, softmax_scale, causal, workspace, workspace_bytes, dev_error, stream, &fs);
 }
 
 pa_status pa_selftest_bounded_wait(int32_t *dev_error, int64_t max_polls, void *stream) {

@@ -89,12 +89,21 @@ struct PrefillArgs {
     int32_t key_chunk, nchunks;         // non-causal: split the keys into chunks of key_chunk (0: one chunk)
     float *part_o, *part_lse;           // non-NULL: write fp32 partials [row, head, part_slots, D] + lse
     int32_t part_slots, part_base;      // partial slots per (row, head); first slot used by chunk 0
+    // --- pa_store_kv_prefill_varlen (NULL new_slots otherwise): the new keys come from the new K/V rows
+    // (row cu_q[s] + i is key c + i of sequence s), which are also stored to their cache slots ---
+    const void *k_new, *v_new;
+    int64_t kn_stride, vn_stride;       // elements
+    const int32_t *new_slots;           // [total_q]
+    void *k_cache, *v_cache;
+    int64_t num_slots;
 };
 size_t prefill_workspace_bytes(int32_t batch, int32_t max_seqlen_q, int32_t group, int32_t num_kv_heads,
                                int32_t nchunks = 1);
 constexpr int32_t kPrefillMaxBatch = 6144;   // the planning kernel keeps 2 ints per sequence in shared memory
+// tm_kn / tm_vn: maps of the new K/V rows, required when a.new_slots is set (ignored otherwise)
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
-                           const CUtensorMap &tm_v, cudaStream_t stream);
+                           const CUtensorMap &tm_v, cudaStream_t stream, const CUtensorMap *tm_kn = nullptr,
+                           const CUtensorMap *tm_vn = nullptr);
 
 // ------------------------------------------------------------ error text --
 // Record the text pa_last_error_detail() returns on this thread.

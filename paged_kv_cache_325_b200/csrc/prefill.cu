@@ -54,17 +54,22 @@ constexpr int kSlab = kM * kRowBytes;  // 128 rows x 128 B = 16 KB
 constexpr int kUnitQueue = 4;          // unit ids handed from the TMA warp to the other roles
 constexpr int kPlanThreads = 1024;
 
-template <int D>
+// kFused: the store fused in (pa_store_kv_prefill_varlen) needs a staging area for the rows it copies; at
+// D = 128 it takes the room of one K/V ring slot.
+template <int D, bool kFused = false>
 struct PrefillCfg {
     static constexpr int kHalves = D / 64;
-    static constexpr int kSlots = D == 128 ? 5 : 8;             // K/V ring slots (one K or V tile each)
+    static constexpr int kSlots = D == 128 ? (kFused ? 4 : 5) : 8;   // K/V ring slots (one K or V tile each)
     static constexpr int kTileBytes = kHalves * kSlab;          // a Q tile, or a K or V tile of 128 keys
     static constexpr int kQOff = 0;                             // Q_A, Q_B
     static constexpr int kRingOff = kQOff + 2 * kTileBytes;
-    static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
+    static constexpr int kStageTokens = 64;                     // fused store: rows per copy round
+    static constexpr int kStageOff = kRingOff + kSlots * kTileBytes;   // [token][K row, V row]
+    static constexpr int kStageBytes = kFused ? kStageTokens * 4 * D : 0;
+    static constexpr int kBarOff = kStageOff + kStageBytes;
     // kv_full[S] kv_empty[S] q_full q_empty s_full[2] p_full[2] o_full[2] o_empty[2] done uq_full[4] uq_empty[4]
-    // v_fixed vlast_full[2]
-    static constexpr int kNumBars = 2 * kSlots + 11 + 2 * kUnitQueue + 3;
+    // v_fixed vlast_full[2] cp_full
+    static constexpr int kNumBars = 2 * kSlots + 11 + 2 * kUnitQueue + 3 + 1;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 64 + kUnitQueue * 64 + 1024;
     static constexpr uint32_t kTmemCols = 512;                  // S_A 0, O_A 128, S_B 256, O_B 384
                                                                 // (P_X, bf16, overwrites the first 64 columns of S_X)
@@ -256,11 +261,14 @@ __global__ void __launch_bounds__(kPlanThreads)
     }
 }
 
-template <int D>
+// kFused: pa_store_kv_prefill_varlen.  Keys past the cached prefix come from the new K/V rows (tm_kn, tm_vn)
+// instead of the cache, and the V-fix warp stores each unit's own new rows to their cache slots.
+template <int D, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
-    using C = PrefillCfg<D>;
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kn,
+                   const __grid_constant__ CUtensorMap tm_vn, const PrefillArgs a) {
+    using C = PrefillCfg<D, kFused>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
@@ -280,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // one unit ahead of the V-fix warp (the next unit's loads wait for this unit's S products, and those
     // wait for the fix), so two barriers keep every phase distinct.
     uint64_t *vlast_full = v_fixed + 1;           // [2]
+    uint64_t *cp_full = vlast_full + 2;           // fused store: a copy round's rows are in the staging area
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
     // unit queue: kUnitQueue entries of 16 words (a decoded Unit; valid = -1 ends the stream)
     volatile int32_t *unit_q = reinterpret_cast<volatile int32_t *>(tmem_slot + 16);
@@ -311,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(smem_u32(v_fixed), 1);
         mbar_init(smem_u32(vlast_full), 1);
         mbar_init(smem_u32(vlast_full + 1), 1);
+        mbar_init(smem_u32(cp_full), 1);
         for (int i = 0; i < kUnitQueue; ++i) {
             mbar_init(smem_u32(uq_full + i), 1);
             mbar_init(smem_u32(uq_empty + i), 10);  // the MMA warp, the V-fix warp, the eight softmax warps
@@ -432,7 +442,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int blk = __shfl_sync(0xffffffffu, ids, tok / B - chunk);
                             if (lane == 0) {
                                 int row;
-                                if ((unsigned)blk < (unsigned)a.num_blocks) {
+                                const CUtensorMap *map = kv ? &tm_v : &tm_k;
+                                if (kFused && tok >= U.c) {
+                                    // a new key: row q0 + (tok - c) of the new K/V (a box never straddles c,
+                                    // which is a whole number of blocks); rows past the tensor read zeros
+                                    row = U.q0 + (tok - U.c);
+                                    map = kv ? &tm_vn : &tm_kn;
+                                } else if ((unsigned)blk < (unsigned)a.num_blocks) {
                                     row = blk * B + (tok % B);
                                 } else {
                                     report(a.dev_error, PA_DEVERR_BLOCK_ID);
@@ -440,8 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 }
 #pragma unroll
                                 for (int h = 0; h < C::kHalves; ++h)
-                                    tma_load_3d(dst + h * kSlab + b * box * kRowBytes, kv ? &tm_v : &tm_k, h * 64,
-                                                U.kvh, row, fb);
+                                    tma_load_3d(dst + h * kSlab + b * box * kRowBytes, map, h * 64, U.kvh, row, fb);
                             }
                         }
                     }
@@ -566,14 +581,122 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ========================================================== V fix ==
         // Zero the rows of each unit's last V tile past its key range (stale or poisoned cache slots),
         // so that masked keys, whose probabilities are exactly 0, never meet a NaN.
+        // Fused store: between those fixes this warp copies each unit's own new tokens' K/V rows of its KV
+        // head to their cache slots with the bulk-copy engine, in rounds of up to kStageTokens tokens:
+        // bulk loads of the rows into the staging area (completing on cp_full), then one bulk store per
+        // row to its slot.  The warp never waits on a copy while a fix is due -- it polls for the next
+        // unit's last V tile between steps -- so the MMA waits for fixes only.  Units whose rows are not
+        // yet copied wait in a small FIFO; the rest is copied when the CTA has no unit left.  No kernel of
+        // this launch reads those slots.
         uint32_t L = 0, nfx = 0;
+        constexpr int kFifo = 4;
+        int fq_s[kFifo], fq_kvh[kFifo], fq_q0[kFifo], fq_c[kFifo], fq_i[kFifo], fq_end[kFifo];
+        int fq_head = 0, fq_n = 0;            // oldest entry, entries in use
+        int cp_state = 0;                     // 0: staging free, 1: loads in flight, 2: stores issued
+        uint32_t cp_rounds = 0;               // completed phases of cp_full
+        int rd_s = 0, rd_kvh = 0, rd_q0 = 0, rd_c = 0, rd_i = 0, rd_n = 0;   // the round in flight
+        const uint32_t stage = sbase + C::kStageOff;
+        const uint32_t cpb = smem_u32(cp_full);
+        // take up to kStageTokens tokens of the oldest pending unit and start their loads
+        auto start_round = [&]() {
+            int end = 0;
+#pragma unroll
+            for (int e = 0; e < kFifo; ++e)
+                if (e == fq_head) {
+                    rd_s = fq_s[e];
+                    rd_kvh = fq_kvh[e];
+                    rd_q0 = fq_q0[e];
+                    rd_c = fq_c[e];
+                    rd_i = fq_i[e];
+                    end = fq_end[e];
+                }
+            rd_n = min(C::kStageTokens, end - rd_i);
+#pragma unroll
+            for (int e = 0; e < kFifo; ++e)
+                if (e == fq_head) fq_i[e] = rd_i + rd_n;
+            if (rd_i + rd_n >= end) {
+                fq_head = (fq_head + 1) % kFifo;
+                --fq_n;
+            }
+            if (lane == 0) mbar_arrive_expect_tx(cpb, (uint32_t)(rd_n * 4 * D));
+            __syncwarp();
+            for (int t = lane; t < rd_n; t += 32) {
+                const int64_t row = (int64_t)rd_q0 + rd_i + t;
+                bulk_load(stage + t * 4 * D,
+                          static_cast<const __nv_bfloat16 *>(a.k_new) + row * a.kn_stride + (int64_t)rd_kvh * D, 2 * D,
+                          cpb);
+                bulk_load(stage + t * 4 * D + 2 * D,
+                          static_cast<const __nv_bfloat16 *>(a.v_new) + row * a.vn_stride + (int64_t)rd_kvh * D, 2 * D,
+                          cpb);
+            }
+            cp_state = 1;
+        };
+        // the round's rows have landed: one bulk store per row to its slot
+        auto store_round = [&]() {
+            mbar_wait(cpb, cp_rounds & 1, a.dev_error);   // returns at once: every lane acquires the rows
+            ++cp_rounds;
+            for (int t = lane; t < rd_n; t += 32) {
+                const int64_t row = (int64_t)rd_q0 + rd_i + t;
+                const int32_t sl = __ldg(a.new_slots + row);
+                if (sl < 0 || (int64_t)sl >= a.num_slots) {
+                    report(a.dev_error, PA_DEVERR_SLOT);   // not stored
+                    continue;
+                }
+                if (a.dev_error) {   // the slot must be the row this prefill read as key c + i
+                    const int pos = rd_c + rd_i + t;
+                    const int32_t blk = __ldg(a.block_table + (int64_t)rd_s * a.bt_stride + pos / a.block_size);
+                    if ((int64_t)sl != (int64_t)blk * a.block_size + pos % a.block_size) report(a.dev_error, PA_DEVERR_SLOT);
+                }
+                const int64_t off = ((int64_t)sl * a.num_kv_heads + rd_kvh) * D;
+                bulk_store(static_cast<__nv_bfloat16 *>(a.k_cache) + off, stage + t * 4 * D, 2 * D);
+                bulk_store(static_cast<__nv_bfloat16 *>(a.v_cache) + off, stage + t * 4 * D + 2 * D, 2 * D);
+            }
+            bulk_commit();
+            cp_state = 2;
+        };
+        // One loop, one site for each copy step.  With no unit left it drains the FIFO.
+        bool more = true;
         for (uint32_t k = 0;; ++k) {
             Unit U;
-            if (!pop_unit(k, lane == 0, U)) break;
-            if (!U.valid) continue;
+            U.valid = 0;
+            if (more && !pop_unit(k, lane == 0, U)) more = false;
+            if (more && !U.valid) continue;
+            const uint32_t vbar = smem_u32(vlast_full + (nfx & 1)), vpar = (nfx >> 1) & 1;
+            if (kFused) {
+                // pump the copy engine until the unit's last V tile lands (a fix first, always) or, with
+                // no unit left, until nothing is pending; leave room in the FIFO for this unit.  Bounded:
+                // polls sleep 128 ns and a round's loads are waited for at most kWaitTimeoutNs.
+                uint64_t t_loads = 0;
+                for (;;) {
+                    if (more && fq_n < kFifo && __any_sync(0xffffffffu, mbar_test_wait(vbar, vpar))) break;
+                    if (cp_state == 1) {
+                        const bool landed = __any_sync(0xffffffffu, mbar_test_wait(cpb, cp_rounds & 1));
+                        if (landed || !more || (t_loads && global_timer_ns() - t_loads > kWaitTimeoutNs)) {
+                            store_round();
+                            t_loads = 0;
+                        } else {
+                            if (!t_loads) t_loads = global_timer_ns();
+                            __nanosleep(128);
+                        }
+                        continue;
+                    }
+                    if (cp_state == 2) {          // the staging area is free once the stores have read it
+                        bulk_wait_read();
+                        __syncwarp();
+                        cp_state = 0;
+                        continue;
+                    }
+                    if (fq_n > 0) {
+                        start_round();
+                        continue;
+                    }
+                    break;                        // nothing pending
+                }
+            }
+            if (!more) break;
             const uint32_t vidx = L + 2 * (U.nk - 1) + 1;
             L += 2 * U.nk;
-            if (!mbar_wait(smem_u32(vlast_full + (nfx & 1)), (nfx >> 1) & 1, a.dev_error)) break;
+            if (!mbar_wait(vbar, vpar, a.dev_error)) break;
             ++nfx;
             const int valid = max(U.kend[0], U.kend[1]) - (U.kbeg + (U.nk - 1) * kN);
             if (valid < kN) {
@@ -589,6 +712,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(v_fixed));
+            if (kFused && U.chunk == 0) {
+                // this unit's own tokens: tile A's, then tile B's (present only when tile A is full); the
+                // loop above left room in the FIFO
+                const int e_new = (fq_head + fq_n) % kFifo;
+                const int i0 = U.tok0[0], i1 = min(U.n_new, U.tok0[0] + 2 * TQ);
+#pragma unroll
+                for (int e = 0; e < kFifo; ++e)
+                    if (e == e_new) {
+                        fq_s[e] = U.s;
+                        fq_kvh[e] = U.kvh;
+                        fq_q0[e] = U.q0;
+                        fq_c[e] = U.c;
+                        fq_i[e] = i0;
+                        fq_end[e] = i1;
+                    }
+                if (i1 > i0) ++fq_n;
+            }
+        }
+        if (kFused) {
+            // leave nothing in flight: the last round's loads (bounded), then every bulk store
+            if (cp_state == 1) mbar_wait(cpb, cp_rounds & 1, a.dev_error);
+            bulk_wait_all();
         }
     } else {
         // ======================================================== softmax ==
@@ -734,17 +879,20 @@ int num_sms() {
 
 template <int D>
 cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
-                             const CUtensorMap &tm_v, cudaStream_t stream) {
-    using C = PrefillCfg<D>;
-    static std::atomic<uint64_t> configured{0};
+                             const CUtensorMap &tm_v, const CUtensorMap &tm_kn, const CUtensorMap &tm_vn,
+                             cudaStream_t stream) {
+    const bool fused = a.new_slots != nullptr;
+    auto kernel = fused ? prefill_kernel<D, true> : prefill_kernel<D, false>;
+    const int smem_bytes = fused ? PrefillCfg<D, true>::kSmemBytes : PrefillCfg<D, false>::kSmemBytes;
+    static std::atomic<uint64_t> configured[2] = {{0}, {0}};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const uint64_t bit = uint64_t(1) << (dev & 63);
-    if (!(configured.load(std::memory_order_acquire) & bit)) {
-        e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (!(configured[fused].load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
         if (e != cudaSuccess) return e;
-        configured.fetch_or(bit, std::memory_order_acq_rel);
+        configured[fused].fetch_or(bit, std::memory_order_acq_rel);
     }
     const int TQ = kM / a.group;
     const size_t plan_smem = (size_t)2 * a.batch * sizeof(int32_t);
@@ -757,14 +905,14 @@ cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &tm_q, cons
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.dynamicSmemBytes = smem_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_kernel<D>, tm_q, tm_k, tm_v, a);
+    return cudaLaunchKernelEx(&cfg, kernel, tm_q, tm_k, tm_v, tm_kn, tm_vn, a);
 }
 
 }  // namespace
@@ -779,9 +927,12 @@ size_t prefill_workspace_bytes(int32_t batch, int32_t max_seqlen_q, int32_t grou
 }
 
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
-                           const CUtensorMap &tm_v, cudaStream_t stream) {
-    if (a.head_dim == 128) return launch_prefill_d<128>(a, tm_q, tm_k, tm_v, stream);
-    return launch_prefill_d<64>(a, tm_q, tm_k, tm_v, stream);
+                           const CUtensorMap &tm_v, cudaStream_t stream, const CUtensorMap *tm_kn,
+                           const CUtensorMap *tm_vn) {
+    if (a.new_slots && (!tm_kn || !tm_vn)) return cudaErrorInvalidValue;
+    const CUtensorMap &kn = tm_kn ? *tm_kn : tm_k, &vn = tm_vn ? *tm_vn : tm_v;   // unused unless fused
+    if (a.head_dim == 128) return launch_prefill_d<128>(a, tm_q, tm_k, tm_v, kn, vn, stream);
+    return launch_prefill_d<64>(a, tm_q, tm_k, tm_v, kn, vn, stream);
 }
 
 }  // namespace pa

@@ -108,6 +108,28 @@ def test_store_decode_validation(lib):
     assert _store_decode(lib, maxc=32768, batch=8) == pa.PA_ERR_WORKSPACE
 
 
+def _store_prefill(lib, **kw):
+    a = dict(k=A, v=A, ks=1024, vs=1024, slots=A, out=A, q=A, tq=150, kc=A, vc=A, cq=A, ck=A, mq=100, mk=200, bt=A,
+             bts=4, batch=2, Hq=32, Hkv=8, D=128, nb=16, B=256, scale=0.088, causal=1, ws=A, wsb=1 << 20, err=None)
+    a.update(kw)
+    return lib.pa_store_kv_prefill_varlen(a["k"], a["v"], a["ks"], a["vs"], a["slots"], a["out"], a["q"], a["tq"],
+                                          a["kc"], a["vc"], a["cq"], a["ck"], a["mq"], a["mk"], a["bt"], a["bts"],
+                                          a["batch"], a["Hq"], a["Hkv"], a["D"], a["nb"], a["B"], a["scale"],
+                                          a["causal"], a["ws"], a["wsb"], a["err"], None)
+
+
+def test_store_prefill_validation(lib):
+    assert _store_prefill(lib, k=None) == pa.PA_ERR_INVALID_ARG
+    assert _store_prefill(lib, slots=None) == pa.PA_ERR_INVALID_ARG
+    assert _store_prefill(lib, vs=1000) == pa.PA_ERR_INVALID_ARG            # shorter than one row
+    assert _store_prefill(lib, ks=1028) == pa.PA_ERR_UNSUPPORTED            # rows not 16-byte aligned
+    assert _store_prefill(lib, k=MIS) == pa.PA_ERR_UNSUPPORTED
+    assert "pa_store_kv then pa_prefill_varlen" in lib.pa_last_error_detail().decode()
+    assert _store_prefill(lib, Hq=48, Hkv=8) == pa.PA_ERR_UNSUPPORTED        # group 6 does not divide 128
+    assert _store_prefill(lib, tq=0) == pa.PA_OK                              # nothing to do
+    assert _store_prefill(lib, ws=None, wsb=0) == pa.PA_ERR_WORKSPACE
+
+
 def test_decode_workspace_size_query():
     assert pa.pa_decode_workspace_size(0, 32, 8, 128, 32768, 256) == 0
     n = pa.pa_decode_workspace_size(8, 32, 8, 128, 32768, 256)

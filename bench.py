@@ -382,6 +382,8 @@ def bench_secondary(args, device, pk, names):
         torch.cuda.empty_cache()
     if "block_size_sweep" in names:
         out["block_size_sweep"] = block_size_sweep(device, pk, timer, steps)
+    if "mixed_batch" in names:
+        out["mixed_batch"] = mixed_batch(device, timer, steps)
     if "varlen_prefill" not in names:
         return out
     case = W.varlen_prefill(poison=False, keep_contiguous=False)
@@ -429,6 +431,45 @@ def bench_secondary(args, device, pk, names):
                      "traffic": recorded_traffic("prefill_varlen")},
     }
     return out
+
+
+def mixed_batch(device, timer, steps):
+    """A step that mixes 64 decode rows (one new token after 512..4096 cached tokens) with 4 prompts of
+    512 new tokens, Qwen3-class heads (32 q / 8 kv, D 128, B 256): the whole batch through the prefill
+    kernel (pa_prefill_varlen) against the one-token rows routed to the decode kernel
+    (pa_prefill_varlen_mixed).  The store of the step's rows is done before, outside the timing."""
+    import paged_kv_cache_325_b200 as pa
+    from paged_kv_cache_325_b200 import workloads as W
+    rng = np.random.Generator(np.random.PCG64(1006))
+    blocks = rng.integers(2, 17, size=64)
+    L = [int(b) * 256 + 1 for b in blocks] + [512] * 4
+    c = [int(b) * 256 for b in blocks] + [0] * 4
+    case = W.make_prefill_case(L, c, 32, 8, 128, 256, seed=2006, poison=False, keep_contiguous=False)
+    dev = device
+    kc, vc, q = case.k_cache.to(dev), case.v_cache.to(dev), case.q.to(dev)
+    bt = torch.as_tensor(case.block_table).to(dev)
+    cq = torch.as_tensor(case.cu_seqlens_q).to(dev)
+    ck = torch.as_tensor(case.cu_seqlens_k).to(dev)
+    o = torch.empty_like(q)
+    pa.pa_store_kv(case.k_new.to(dev), case.v_new.to(dev), torch.as_tensor(case.slot_mapping).to(dev), kc, vc)
+    pws = pa.alloc_prefill_workspace(q, 8, case.batch, case.max_seqlen_q)
+    mws = pa.alloc_mixed_workspace(q, 8, case.batch, case.max_seqlen_q, case.max_seqlen_k)
+
+    def pf():
+        pa.pa_prefill_varlen(o, q, kc, vc, cq, ck, case.max_seqlen_q, case.max_seqlen_k, bt, case.softmax_scale,
+                             workspace=pws)
+
+    def mx():
+        pa.pa_prefill_varlen_mixed(o, q, kc, vc, cq, ck, case.max_seqlen_q, case.max_seqlen_k, bt,
+                                   case.softmax_scale, workspace=mws)
+
+    r1, _g1 = capture(pf)
+    r2, _g2 = capture(mx)
+    timer.run([r1, r2], 5)
+    t1, t2 = timer.run([r1, r2], steps)
+    del r1, r2, _g1, _g2
+    return {"decode_rows": 64, "prompt_tokens": 4 * 512, "prefill_kernel_only_us": statistics.mean(t1) * 1e6,
+            "routed_us": statistics.mean(t2) * 1e6}
 
 
 def block_size_sweep(device, pk, timer, steps):
@@ -547,7 +588,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
-    ap.add_argument("--secondary", default="long_context_decode,prefix_sharing_decode,varlen_prefill",
+    ap.add_argument("--secondary", default="long_context_decode,prefix_sharing_decode,varlen_prefill,mixed_batch",
                     help="comma list of extra workloads to time at N=1 ('none' for none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -315,6 +315,29 @@ PA_API pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, co
                             void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream);
 
 /*
+ * pa_prefill_varlen_mixed -- pa_prefill_varlen for a batch that mixes prompts
+ * with decode steps (the pages' per-step context carries both cu_seqlens_q/k
+ * and context_lens; nano-vllm walkthrough, section eight).  Sequences with
+ * exactly one new token are computed by the split-KV decode kernel (their q /
+ * out row is cu_seqlens_q[s], their context n_k), the others by the prefill
+ * kernel, both in this call and on `stream`.  The result is the function
+ * pa_prefill_varlen computes (causal); only the kernels differ: a one-token
+ * row in the prefill kernel costs a 128-row tile of the tensor cores, in the
+ * decode kernel one pass over its keys.  Arguments as pa_prefill_varlen
+ * (always causal); workspace: pa_prefill_varlen_mixed_workspace_size() bytes,
+ * 256-byte aligned, no initialisation needed.
+ */
+PA_API size_t pa_prefill_varlen_mixed_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim);
+PA_API pa_status pa_prefill_varlen_mixed(void *out, const void *q, int32_t total_q, const void *k_cache,
+                                         const void *v_cache, const int32_t *cu_seqlens_q,
+                                         const int32_t *cu_seqlens_k, int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                         const int32_t *block_table, int32_t block_table_stride, int32_t batch,
+                                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t num_blocks, int32_t block_size, float softmax_scale,
+                                         void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream);
+
+/*
  * pa_store_kv_prefill_varlen -- pa_store_kv of the prompts' new K/V rows
  * followed by pa_prefill_varlen, in one launch, with the new keys read
  * straight from the new K/V rows instead of back from the cache (the prefill

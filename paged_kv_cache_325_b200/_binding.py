@@ -33,7 +33,8 @@ PA_DEVERR_SEQLENS = 0x8
 PA_DEVERR_TIMEOUT = 0x10
 
 __all__ = ["PagedAttnError", "load_library", "declared_symbols", "pa_store_kv", "pa_decode", "pa_decode_split",
-           "pa_store_kv_decode", "pa_store_kv_prefill_varlen",
+           "pa_store_kv_decode", "pa_store_kv_prefill_varlen", "pa_prefill_varlen_mixed",
+           "pa_prefill_varlen_mixed_workspace_size", "alloc_mixed_workspace",
            "pa_decode_workspace_size", "pa_decode_split_workspace_size", "pa_decode_noalloc",
            "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size", "alloc_shared_prefix_workspace", "pa_prefill_varlen",
            "pa_prefill_workspace_size", "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
@@ -77,6 +78,10 @@ _SIGS = {
     "pa_store_kv_prefill_varlen": (ctypes.c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p, _c_i32, _c_p, _c_p,
                                                   _c_p, _c_p, _c_i32, _c_i32, _c_p, _c_i32, _c_i32, _c_i32, _c_i32,
                                                   _c_i32, _c_i32, _c_i32, _c_f32, _c_i32, _c_p, _c_sz, _c_p, _c_p]),
+    "pa_prefill_varlen_mixed_workspace_size": (_c_sz, [_c_i32] * 6),
+    "pa_prefill_varlen_mixed": (ctypes.c_int, [_c_p, _c_p, _c_i32, _c_p, _c_p, _c_p, _c_p, _c_i32, _c_i32, _c_p,
+                                               _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_f32, _c_p,
+                                               _c_sz, _c_p, _c_p]),
     "pa_selftest_bounded_wait": (ctypes.c_int, [_c_p, _c_i64, _c_p]),
 }
 
@@ -367,6 +372,44 @@ def pa_store_kv_prefill_varlen(k, v, slot_mapping, out, q, k_cache, v_cache, cu_
         _ptr(v_cache), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), int(max_seqlen_q), int(max_seqlen_k),
         _ptr(block_table), block_table.shape[1], batch, q.shape[1], Hkv, D, nb, B, float(softmax_scale),
         int(bool(causal)), _ptr(workspace), ws, _opt_err(dev_error, dev), _stream(q, stream)))
+
+
+def pa_prefill_varlen_mixed_workspace_size(batch, max_seqlen_q, max_seqlen_k, num_q_heads, num_kv_heads,
+                                           head_dim) -> int:
+    return int(load_library().pa_prefill_varlen_mixed_workspace_size(batch, max_seqlen_q, max_seqlen_k, num_q_heads,
+                                                                     num_kv_heads, head_dim))
+
+
+def alloc_mixed_workspace(q, num_kv_heads, batch, max_seqlen_q, max_seqlen_k):
+    """A torch-owned workspace of the size pa_prefill_varlen_mixed needs."""
+    import torch
+    n = pa_prefill_varlen_mixed_workspace_size(batch, max_seqlen_q, max_seqlen_k, q.shape[1], num_kv_heads,
+                                               q.shape[2])
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+
+
+def pa_prefill_varlen_mixed(out, q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                            block_table, softmax_scale, workspace=None, dev_error=None, stream=None):
+    """Causal varlen attention for a batch mixing prompts and decode steps (one-token sequences go to the
+    decode kernel, the rest to the prefill kernel)."""
+    import torch
+    nb, B, Hkv, D = _cache_dims(k_cache, v_cache)
+    dev = k_cache.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(out, "out", torch.bfloat16, dev)
+    if q.dim() != 3 or q.shape[2] != D or out.shape != q.shape:
+        raise ValueError("q and out must be [total_q, num_q_heads, head_dim]")
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, dev)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, dev)
+    _need(block_table, "block_table", torch.int32, dev)
+    batch = int(cu_seqlens_q.shape[0]) - 1
+    if cu_seqlens_k.shape != cu_seqlens_q.shape or block_table.dim() != 2 or block_table.shape[0] != batch:
+        raise ValueError("cu_seqlens_q/k must be [batch+1] and block_table [batch, max_blocks]")
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load_library().pa_prefill_varlen_mixed(
+        _ptr(out), _ptr(q), int(q.shape[0]), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+        int(max_seqlen_q), int(max_seqlen_k), _ptr(block_table), block_table.shape[1], batch, q.shape[1], Hkv, D,
+        nb, B, float(softmax_scale), _ptr(workspace), ws, _opt_err(dev_error, dev), _stream(q, stream)))
 
 
 def pa_selftest_bounded_wait(dev_error, max_polls, stream=None):

@@ -91,9 +91,23 @@ constexpr int kPlanHdrBytes = 256;
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBuckets = 1024;          // item lengths (tiles) for the longest-first order; longer share the last
 
+// Context length of sequence s: context_lens[s]; in the varlen mode (the decode rows of a mixed batch) the
+// key count of a sequence with exactly one new token, and -1 for any other sequence (not this call's work).
+__device__ __forceinline__ int dec_ctx(const DecodeArgs &a, int s) {
+    if (!a.vl_cu_q) return __ldg(a.context_lens + s);
+    if (__ldg(a.vl_cu_q + s + 1) - __ldg(a.vl_cu_q + s) != 1) return -1;
+    return __ldg(a.vl_cu_k + s + 1) - __ldg(a.vl_cu_k + s);
+}
+
+// Row of sequence s in q and out.
+__device__ __forceinline__ int64_t dec_row(const DecodeArgs &a, int s) {
+    return a.vl_cu_q ? (int64_t)__ldg(a.vl_cu_q + s) : (int64_t)s;
+}
+
 // Item: {s, kvh | split << 16, t_begin, t_end}; s < 0 marks the end of the stream in shared memory.
 __device__ __forceinline__ int dec_tiles(const DecodeArgs &a, int s, bool report_bad) {
-    const int ctx = __ldg(a.context_lens + s);
+    const int ctx = dec_ctx(a, s);
+    if (ctx == -1) return 0;                  // a prefill sequence of a mixed batch
     if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size ||
         ctx < a.t_offset) {
         if (report_bad) report(a.dev_error, PA_DEVERR_CONTEXT_LEN);
@@ -194,7 +208,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         const int tiles = dec_tiles(a, s, false);
         const int n = dec_nsplit(tiles, whole, chunk);
         if (n == 0) continue;
-        const int ctx = __ldg(a.context_lens + s);
+        const int ctx = dec_ctx(a, s);
         if (n == 1) {
             items[atomicAdd(&s_off[bucket(tiles)], 1)] = make_int4(s, kvh, a.t_offset, ctx);
             continue;
@@ -297,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const uint32_t qbytes = (uint32_t)(G * D * 2);
                 mbar_arrive_expect_tx(smem_u32(qfull + qs), qbytes);
                 bulk_load(qsm + qs * qslot,
-                          static_cast<const __nv_bfloat16 *>(a.q) + ((int64_t)s * a.num_q_heads + (int64_t)kvh * G) * D,
+                          static_cast<const __nv_bfloat16 *>(a.q) + (dec_row(a, s) * a.num_q_heads + (int64_t)kvh * G) * D,
                           qbytes, smem_u32(qfull + qs));
                 ++nqi;
                 const int32_t *bt = a.block_table + (int64_t)s * a.bt_stride;
@@ -368,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         it.t_begin = d.z;
         it.t_end = d.w;
         it.ntiles = (it.t_end - it.t_begin + kTile - 1) / kTile;
-        it.ctx = __ldg(a.context_lens + it.s);
+        it.ctx = dec_ctx(a, it.s);
         // fused store: this warp owns the new token's row if position ctx - 1 falls in its slice of the
         // pair's last split; the row is staged now and used when its tile lands
         // own: 0, or 1 (this warp stores the new row) | 2 (the slot is the row this decode reads: the tile is
@@ -591,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             const int h = it.kvh * G + g;
             if (direct) {
-                static_cast<__nv_bfloat16 *>(a.out)[((int64_t)it.s * a.num_q_heads + h) * D + d] =
+                static_cast<__nv_bfloat16 *>(a.out)[(dec_row(a, it.s) * a.num_q_heads + h) * D + d] =
                     __float2bfloat16_rn(ot / lt);
             } else {
                 const int64_t pi = ((int64_t)it.s * a.num_q_heads + h) * a.part_slots + a.part_base + it.split;
@@ -612,7 +626,7 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
     asm volatile("griddepcontrol.wait;" ::: "memory");   // partials of the split kernel are visible
     const int h = blockIdx.x % a.num_q_heads;
     const int s = blockIdx.x / a.num_q_heads;
-    const int ctx = __ldg(a.context_lens + s);
+    const int ctx = dec_ctx(a, s);              // -1: not this call's work
     if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size ||
         ctx < a.t_offset)
         return;
@@ -644,7 +658,7 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den_lane += __shfl_xor_sync(0xffffffffu, den_lane, o);
-    static_cast<__nv_bfloat16 *>(a.out)[((int64_t)s * a.num_q_heads + h) * D + d] =
+    static_cast<__nv_bfloat16 *>(a.out)[(dec_row(a, s) * a.num_q_heads + h) * D + d] =
         __float2bfloat16_rn(num / den_lane);
 }
 

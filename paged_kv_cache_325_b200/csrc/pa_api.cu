@@ -495,7 +495,7 @@ static pa_status prefill_impl(void *out, const void *q, int32_t total_q, const v
                               int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                               int32_t num_blocks, int32_t block_size, float softmax_scale, int32_t causal,
                               void *workspace, size_t workspace_bytes, int32_t *dev_error, void *stream,
-                              const FusedStore *fs) {
+                              const FusedStore *fs, int32_t skip_single = 0) {
     if (batch < 0) return fail(PA_ERR_INVALID_ARG, "batch < 0");
     pa_status st = check_cache_shape(num_blocks, block_size, num_kv_heads, head_dim);
     if (st != PA_OK) return st;
@@ -562,6 +562,7 @@ static pa_status prefill_impl(void *out, const void *q, int32_t total_q, const v
     a.nchunks = 1;
     a.part_o = a.part_lse = nullptr;
     a.part_slots = a.part_base = 0;
+    a.skip_single = skip_single;
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
 
     CUtensorMap tm_k, tm_v;
@@ -605,6 +606,90 @@ pa_status pa_prefill_varlen(void *out, const void *q, int32_t total_q, const voi
     return prefill_impl(out, q, total_q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
                         block_table, block_table_stride, batch, num_q_heads, num_kv_heads, head_dim, num_blocks,
                         block_size, softmax_scale, causal, workspace, workspace_bytes, dev_error, stream, nullptr);
+}
+
+size_t pa_prefill_varlen_mixed_workspace_size(int32_t batch, int32_t max_seqlen_q, int32_t max_seqlen_k,
+                                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim) {
+    if (batch <= 0 || max_seqlen_q <= 0 || max_seqlen_k <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+        num_q_heads % num_kv_heads != 0 || 128 % (num_q_heads / num_kv_heads) != 0 || head_dim <= 0)
+        return 0;
+    const size_t pf = (pa::prefill_workspace_bytes(batch, max_seqlen_q, num_q_heads / num_kv_heads, num_kv_heads) +
+                       255) / 256 * 256;
+    const pa::DecodePlan plan = pa::plan_decode(batch, num_kv_heads, max_seqlen_k, 0, num_sms_current());
+    return pf + pa::decode_workspace_layout(plan, batch, num_q_heads, num_kv_heads, head_dim).total;
+}
+
+pa_status pa_prefill_varlen_mixed(void *out, const void *q, int32_t total_q, const void *k_cache, const void *v_cache,
+                                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t max_seqlen_q,
+                                  int32_t max_seqlen_k, const int32_t *block_table, int32_t block_table_stride,
+                                  int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                  int32_t num_blocks, int32_t block_size, float softmax_scale, void *workspace,
+                                  size_t workspace_bytes, int32_t *dev_error, void *stream) {
+    if (batch < 0) return fail(PA_ERR_INVALID_ARG, "batch < 0");
+    if (batch == 0 || max_seqlen_q == 0 || total_q == 0)   // (the prefill call below validates the rest)
+        return prefill_impl(out, q, total_q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                            max_seqlen_k, block_table, block_table_stride, batch, num_q_heads, num_kv_heads, head_dim,
+                            num_blocks, block_size, softmax_scale, 1, workspace, workspace_bytes, dev_error, stream,
+                            nullptr, 1);
+    pa_status st = check_heads(num_q_heads, num_kv_heads);
+    if (st != PA_OK) return st;
+    if (max_seqlen_k < 1 || max_seqlen_q < 0 || head_dim < 1)
+        return fail(PA_ERR_INVALID_ARG, "need max_seqlen_k >= 1 and head_dim >= 1");
+    const size_t need = pa_prefill_varlen_mixed_workspace_size(batch, max_seqlen_q, max_seqlen_k, num_q_heads,
+                                                               num_kv_heads, head_dim);
+    if (need == 0) return fail(PA_ERR_UNSUPPORTED, "shape not supported (the GQA group must divide 128)");
+    if (!workspace || workspace_bytes < need)
+        return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (!aligned(workspace, 256)) return fail(PA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const size_t pf_bytes =
+        (pa::prefill_workspace_bytes(batch, max_seqlen_q, num_q_heads / num_kv_heads, num_kv_heads) + 255) / 256 * 256;
+    // 1. the prompts (every sequence with more than one new token): the prefill kernel; it validates
+    //    every argument before anything is enqueued
+    st = prefill_impl(out, q, total_q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                      block_table, block_table_stride, batch, num_q_heads, num_kv_heads, head_dim, num_blocks,
+                      block_size, softmax_scale, 1, workspace, pf_bytes, dev_error, stream, nullptr, 1);
+    if (st != PA_OK) return st;
+    // 2. the decode rows (one new token, context n_k): the split-KV decode in its varlen mode
+    pa::DecodeArgs da = {};
+    da.plan = pa::plan_decode(batch, num_kv_heads, max_seqlen_k, 0, num_sms_current());
+    if (da.plan.max_splits > pa::kDecodeMaxSplits || num_kv_heads > pa::kDecodeMaxKvHeads)
+        return fail(PA_ERR_UNSUPPORTED, "more than %d context splits or %d KV heads", pa::kDecodeMaxSplits,
+                    pa::kDecodeMaxKvHeads);
+    const pa::DecodeWorkspace wl = pa::decode_workspace_layout(da.plan, batch, num_q_heads, num_kv_heads, head_dim);
+    char *ws = static_cast<char *>(workspace) + pf_bytes;
+    da.plan_ws = ws + wl.plan_off;
+    da.part_o = reinterpret_cast<float *>(ws + wl.o_off);
+    da.part_lse = reinterpret_cast<float *>(ws + wl.lse_off);
+    da.out = out;
+    da.q = q;
+    da.block_table = block_table;
+    da.context_lens = nullptr;
+    da.vl_cu_q = cu_seqlens_q;
+    da.vl_cu_k = cu_seqlens_k;
+    da.dev_error = dev_error;
+    da.bt_stride = block_table_stride;
+    da.batch = batch;
+    da.num_q_heads = num_q_heads;
+    da.num_kv_heads = num_kv_heads;
+    da.group = num_q_heads / num_kv_heads;
+    da.head_dim = head_dim;
+    da.num_blocks = num_blocks;
+    da.block_size = block_size;
+    da.box_tokens = block_size < pa::kDecodeTileTokens ? block_size : pa::kDecodeTileTokens;
+    da.max_context_len = max_seqlen_k;
+    da.scale_log2 = softmax_scale * 1.4426950408889634f;
+    da.part_slots = da.plan.max_splits;
+    da.part_base = 0;
+    da.t_offset = 0;
+    da.num_slots = (int64_t)num_blocks * block_size;
+    CUtensorMap dk, dv;
+    const int64_t rows = (int64_t)num_blocks * block_size;
+    if ((st = encode_rows(&dk, k_cache, rows, num_kv_heads, head_dim, 1, da.box_tokens)) != PA_OK) return st;
+    if ((st = encode_rows(&dv, v_cache, rows, num_kv_heads, head_dim, 1, da.box_tokens)) != PA_OK) return st;
+    cudaError_t e = pa::launch_decode(da, dk, dv, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "mixed-batch decode launch");
+    return ok();
 }
 
 pa_status pa_store_kv_prefill_varlen(const void *k, const void *v, int64_t k_row_stride, int64_t v_row_stride,

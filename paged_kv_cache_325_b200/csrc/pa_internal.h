@@ -62,6 +62,10 @@ struct DecodeArgs {
     int32_t part_slots, part_base;
     int32_t t_offset;        // the split ranges start at this token (shared-prefix decode: P * block_size)
     int32_t shared_blocks;   // checked mode: block_table[s][0..shared_blocks) must equal row 0's
+    // varlen rows (the decode rows of a mixed batch): when set, sequence s is this call's work only if it has
+    // one new token (cu_q[s+1] - cu_q[s] == 1); its q / out row is cu_q[s] and its context cu_k[s+1] - cu_k[s]
+    // (context_lens unused)
+    const int32_t *vl_cu_q, *vl_cu_k;
     // store fused into the decode (pa_store_kv_decode): row s of k_new / v_new is sequence s's new token,
     // written to cache slot new_slots[s] (skipped when < 0); NULL new_slots: no store
     const void *k_new, *v_new;
@@ -89,6 +93,7 @@ struct PrefillArgs {
     int32_t key_chunk, nchunks;         // non-causal: split the keys into chunks of key_chunk (0: one chunk)
     float *part_o, *part_lse;           // non-NULL: write fp32 partials [row, head, part_slots, D] + lse
     int32_t part_slots, part_base;      // partial slots per (row, head); first slot used by chunk 0
+    int32_t skip_single;                // mixed batch: sequences with one new token are the decode's work
     // --- pa_store_kv_prefill_varlen (NULL new_slots otherwise): the new keys come from the new K/V rows
     // (row cu_q[s] + i is key c + i of sequence s), which are also stored to their cache slots ---
     const void *k_new, *v_new;

@@ -181,7 +181,8 @@ __global__ void __launch_bounds__(kPlanThreads)
     for (int s = tid; s < a.batch; s += kPlanThreads) {
         int q0, n_new, n_k;
         if (seq_geometry(a, s, q0, n_new, n_k)) {
-            np[s] = min(R, (n_new + two_tq - 1) / two_tq);
+            // a mixed batch's one-token sequences are the decode kernel's work
+            np[s] = (a.skip_single && n_new == 1) ? 0 : min(R, (n_new + two_tq - 1) / two_tq);
             geo[s] = make_int4(q0, n_new, n_k, 1);
         } else {
             np[s] = 0;

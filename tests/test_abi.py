@@ -130,6 +130,24 @@ def test_store_prefill_validation(lib):
     assert _store_prefill(lib, ws=None, wsb=0) == pa.PA_ERR_WORKSPACE
 
 
+def test_mixed_validation(lib):
+    def call(**kw):
+        a = dict(out=A, q=A, tq=150, kc=A, vc=A, cq=A, ck=A, mq=100, mk=2000, bt=A, bts=8, batch=4, Hq=32, Hkv=8,
+                 D=128, nb=64, B=256, scale=0.088, ws=A, wsb=1 << 26, err=None)
+        a.update(kw)
+        return lib.pa_prefill_varlen_mixed(a["out"], a["q"], a["tq"], a["kc"], a["vc"], a["cq"], a["ck"], a["mq"],
+                                           a["mk"], a["bt"], a["bts"], a["batch"], a["Hq"], a["Hkv"], a["D"], a["nb"],
+                                           a["B"], a["scale"], a["ws"], a["wsb"], a["err"], None)
+    assert call(ws=None, wsb=0) == pa.PA_ERR_WORKSPACE
+    assert call(wsb=256) == pa.PA_ERR_WORKSPACE
+    assert call(Hq=48) == pa.PA_ERR_UNSUPPORTED          # GQA group 6 does not divide 128
+    assert call(Hq=30) == pa.PA_ERR_INVALID_ARG
+    assert call(batch=0) == pa.PA_OK
+    assert call(q=None) == pa.PA_ERR_INVALID_ARG
+    n = pa.pa_prefill_varlen_mixed_workspace_size(4, 100, 2000, 32, 8, 128)
+    assert n >= pa.pa_prefill_workspace_size(4, 100, 32, 8, 128) + pa.pa_decode_workspace_size(4, 32, 8, 128, 2000, 256)
+
+
 def test_decode_workspace_size_query():
     assert pa.pa_decode_workspace_size(0, 32, 8, 128, 32768, 256) == 0
     n = pa.pa_decode_workspace_size(8, 32, 8, 128, 32768, 256)

@@ -197,3 +197,18 @@ def test_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA tensor"):
         pa.pa_decode(q.clone(), q, kc, kc, torch.zeros(2, 1, dtype=torch.int32), torch.ones(2, dtype=torch.int32),
                      1, 0.125)
+
+
+def test_binding_new_entry_points_reject_cpu_tensors():
+    """No CPU path: every entry point refuses host tensors before calling the library."""
+    import torch
+    q = torch.zeros(2, 4, 64, dtype=torch.bfloat16)
+    kv = torch.zeros(2, 2, 64, dtype=torch.bfloat16)
+    kc = torch.zeros(4, 16, 2, 64, dtype=torch.bfloat16)
+    i32 = lambda *shape: torch.zeros(*shape, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        pa.pa_store_kv_decode(kv, kv, i32(2), q.clone(), q, kc, kc, i32(2, 1), i32(2), 16, 0.125)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        pa.pa_store_kv_prefill_varlen(kv, kv, i32(2), q.clone(), q, kc, kc, i32(3), i32(3), 1, 1, i32(2, 1), 0.125)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        pa.pa_prefill_varlen_mixed(q.clone(), q, kc, kc, i32(3), i32(3), 1, 1, i32(2, 1), 0.125)

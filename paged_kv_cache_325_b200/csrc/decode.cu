@@ -37,6 +37,10 @@
 //    writes it into the tile in shared memory (in place of the cache row the
 //    TMA brought) and to its cache slot in HBM -- the store_kvcache of the
 //    walkthrough, section seven, done inside the attention launch.
+//  * varlen mode (pa_prefill_varlen_mixed): the decode rows of a batch that
+//    mixes decode steps with prompts -- sequence s is this call's work only if
+//    it has one new token; its q / out row is cu_seqlens_q[s] and its context
+//    n_k.
 #include <float.h>
 
 #include <atomic>

@@ -15,8 +15,9 @@
 //  * a Q tile is 128 MMA rows = (128 / G) consecutive new tokens x the G
 //    q-heads of one KV head (GQA packing), so one K/V tile feeds all G heads;
 //  * a work unit is two adjacent Q tiles (A, then B) of one (sequence, KV
-//    head); units are ordered by decreasing cost (last tiles of every sequence
-//    first) and dealt round-robin to persistent CTAs, one per SM;
+//    head); a one-CTA planning kernel writes the units into a table ordered by
+//    decreasing cost (last tiles of every sequence first), and persistent CTAs,
+//    one per SM, take them with an atomic counter;
 //  * warp 8 (TMA): per unit, both Q tiles (3-D tensor map over q), then the
 //    K and V tiles of 128 keys, gathered block by block through block_table,
 //    into a ring of shared-memory slots guarded by mbarriers;
@@ -28,12 +29,14 @@
 //  * warps 0-3 / 4-7 (softmax of tile A / B): thread t owns TMEM lane t, i.e.
 //    one Q row; it reads its S row with tcgen05.ld, selects masked keys out
 //    (-inf), keeps a running max in log2 units and rescales O (tcgen05.ld/st)
-//    only when the max grew by more than 8 (2^8), writes P as bf16 into a
-//    swizzled shared-memory tile (the A operand of PV), and after the last key
-//    tile divides O by the row sum and stores bf16 rows;
-//  * V rows of a unit's last key tile beyond its key range are zeroed in
-//    shared memory before the PV products, so stale or poisoned cache contents
-//    never meet a zero weight (0 * NaN is never formed).
+//    only when the max grew by more than 8 (2^8), writes P as packed bf16
+//    back into TMEM over the first columns of its S row (the PV product reads
+//    its A operand from TMEM), and after the last key tile divides O by the
+//    row sum and stores bf16 rows;
+//  * warp 10 (V fix) zeroes the V rows of a unit's last key tile beyond its
+//    key range in shared memory before the PV products, so stale or poisoned
+//    cache contents never meet a zero weight (0 * NaN is never formed); in the
+//    fused-store form it also copies the unit's new K/V rows to their slots.
 #include <atomic>
 
 #include "pa_device.cuh"

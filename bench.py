@@ -47,6 +47,8 @@ PRIMARY_DESC = ("Qwen3-0.6B-like decode layer call: batch 64, context_lens U[100
                 "head_dim 128, block_size 256, shuffled blocks; store of the 64 new K/V rows + paged decode "
                 "(pa_store_kv_decode, one launch)")
 FLUSH_BYTES = 256 << 20
+SECONDARY_STEPS = 50        # timed runs per secondary measurement (median reported)
+CLOCK_SOAK_S = 0.6          # untimed steps on each side of the primary timed region, for the clock sampler
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -177,6 +179,18 @@ def barrier(world):
         dist.barrier()
 
 
+_CASES = {}
+
+
+def get_case(name):
+    """The workload's CPU tensors in their timing form (unused slots filled with N(0,1)), built once and
+    shared by the GPU legs and the CPU-oracle baseline."""
+    from paged_kv_cache_325_b200 import workloads as W
+    if name not in _CASES:
+        _CASES[name] = W.WORKLOADS[name](poison=False, keep_contiguous=False)
+    return _CASES[name]
+
+
 # ----------------------------------------------------------- native timing --
 
 class Timer:
@@ -261,21 +275,37 @@ class DecodeBench:
 
 def bench_primary(args, world, rank, device, pk):
     from paged_kv_cache_325_b200 import workloads as W
-    case = W.WORKLOADS[PRIMARY](poison=False, keep_contiguous=False)
+    case = get_case(PRIMARY)
     b = DecodeBench(case, device)
     # the step: store + decode in one launch (pa_store_kv_decode); the cache rows it writes are the same
     # every step, so every step does the same work
     step_replay, _g0 = capture(b.store_decode)
     timer = Timer(device)
-    timer.run([step_replay], max(args.warmup, 3))
-    barrier(world)
-    torch.cuda.synchronize()
+
+    def soak(seconds):
+        # untimed steps of the same loop (flush + step), so that the clock sampler, whose period is far
+        # longer than the timed region, sees the GPU under this load on both sides of it
+        t_end = time.perf_counter() + seconds
+        while time.perf_counter() < t_end:
+            timer.run([step_replay], 50)
+
     with ClockSampler(local_gpu_index(device)) as clk:
+        t_win = time.perf_counter()
+        timer.run([step_replay], max(args.warmup, 3))
+        soak(CLOCK_SOAK_S)
+        barrier(world)
+        torch.cuda.synchronize()
         (t_step,) = timer.run([step_replay], args.steps)
-    torch.cuda.synchronize()
-    barrier(world)
+        torch.cuda.synchronize()
+        barrier(world)
+        soak(CLOCK_SOAK_S)
+        t_win = time.perf_counter() - t_win
     value, t_max = aggregate(sum(t_step), args.steps * case.batch, world, device)
     step_mean = statistics.mean(t_step)
+    clocks = clk.summary()
+    clocks["window_s"] = round(t_win, 3)
+    clocks["how"] = ("nvidia-smi every 50 ms over a window of the same step loop (L2 flush + graph replay) "
+                     f"that brackets the timed steps: warm-up and {CLOCK_SOAK_S} s of untimed steps on each side")
     alg = b.alg_bytes_decode() + b.alg_bytes_store()
     achieved = alg / step_mean / 1e9
     res = {
@@ -283,24 +313,25 @@ def bench_primary(args, world, rank, device, pk):
         "kv_gbps": case.kv_bytes_read() / step_mean / 1e9,
         "kv_hbm_frac_of_measured": case.kv_bytes_read() / step_mean / 1e9 / pk["hbm_gbs"],
         "kv_hbm_frac_of_8tbs": case.kv_bytes_read() / step_mean / 1e9 / 8000.0,
-        "store_decode_us": step_mean * 1e6,
+        "store_decode_us": step_mean * 1e6, "step_us_median": statistics.median(t_step) * 1e6,
         "roofline": {"kernel": "decode_split_kernel<128> (store fused)", "bound": "hbm",
                      "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                      "traffic": recorded_traffic("store_decode_qwen3_0.6b"), "alg_bytes_per_launch": alg},
         "gpu_launches": 3 * args.steps,     # per step: planning, decode (store fused in) and combine kernels
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
     # the same step as two launches (pa_store_kv, then pa_decode), for comparison; rank 0 at N=1
     if world == 1:
         st_replay, _g1 = capture(b.store)
         dec_replay, _g2 = capture(b.decode)
         timer.run([st_replay, dec_replay], 5)
-        steps2 = max(10, min(args.steps, 500))
+        steps2 = max(SECONDARY_STEPS, min(args.steps, 500))
         t_store, t_dec = timer.run([st_replay, dec_replay], steps2)
-        res["separate_launches"] = {"store_us": statistics.mean(t_store) * 1e6,
-                                    "decode_us": statistics.mean(t_dec) * 1e6,
-                                    "tokens_per_s": case.batch / (statistics.mean(t_store) + statistics.mean(t_dec)),
-                                    "steps": steps2}
+        res["separate_launches"] = {"store_us": statistics.median(t_store) * 1e6,
+                                    "decode_us": statistics.median(t_dec) * 1e6,
+                                    "tokens_per_s": case.batch / (statistics.median(t_store) +
+                                                                  statistics.median(t_dec)),
+                                    "steps": steps2, "statistic": "median"}
     res["e2e"] = bench_e2e(b, args, world, device)
     return case, res
 
@@ -339,15 +370,15 @@ def bench_secondary(args, device, pk, names):
     from paged_kv_cache_325_b200 import workloads as W
     timer = Timer(device)
     out = {}
-    steps = max(10, min(args.steps, 200))
+    steps = SECONDARY_STEPS
     for name in [n for n in names if n in ("long_context_decode", "prefix_sharing_decode")]:
-        case = W.WORKLOADS[name](poison=False, keep_contiguous=False)
+        case = get_case(name)
         b = DecodeBench(case, device)
         b.store()
         dec_replay, _g = capture(b.decode)
         timer.run([dec_replay], 5)
         (t,) = timer.run([dec_replay], steps)
-        tm = statistics.mean(t)
+        tm = statistics.median(t)
         ach = b.alg_bytes_decode() / tm / 1e9
         r = {"decode_us": tm * 1e6, "tokens_per_s": case.batch / tm,
              "kv_gbps_logical": case.kv_bytes_read() / tm / 1e9,
@@ -359,7 +390,7 @@ def bench_secondary(args, device, pk, names):
             r["roofline"] = {"bound": "hbm", "achieved": uniq / tm / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
                              "frac": uniq / tm / 1e9 / pk["hbm_gbs"], "bytes": "unique"}
             (tw,) = timer.run([dec_replay], steps, flush=False)
-            r["decode_us_warm_l2"] = statistics.mean(tw) * 1e6
+            r["decode_us_warm_l2"] = statistics.median(tw) * 1e6
             # the shared-prefix path: the 16 common blocks read once per KV head
             P = case.shared_prefix_blocks
             sws = pa.alloc_shared_prefix_workspace(b.q, case.num_kv_heads, b.mcl, case.block_size, P)
@@ -371,7 +402,7 @@ def bench_secondary(args, device, pk, names):
             sh_replay, _g3 = capture(shared)
             timer.run([sh_replay], 5)
             (ts,) = timer.run([sh_replay], steps)
-            tsm = statistics.mean(ts)
+            tsm = statistics.median(ts)
             r["shared_prefix_path"] = {
                 "decode_us": tsm * 1e6, "tokens_per_s": case.batch / tsm,
                 "kv_gbps_unique": case.kv_bytes_unique() / tsm / 1e9,
@@ -386,7 +417,7 @@ def bench_secondary(args, device, pk, names):
         out["mixed_batch"] = mixed_batch(device, timer, steps)
     if "varlen_prefill" not in names:
         return out
-    case = W.varlen_prefill(poison=False, keep_contiguous=False)
+    case = get_case("varlen_prefill")
     dev = device
     kc, vc = case.k_cache.to(dev), case.v_cache.to(dev)
     kn, vn, q = case.k_new.to(dev), case.v_new.to(dev), case.q.to(dev)
@@ -413,10 +444,10 @@ def bench_secondary(args, device, pk, names):
     fu_replay, _g3 = capture(fused)
     timer.run([st_replay, pf_replay], 5)
     ts, tp = timer.run([st_replay, pf_replay], steps)
-    tpm, tsm = statistics.mean(tp), statistics.mean(ts)
+    tpm, tsm = statistics.median(tp), statistics.median(ts)
     timer.run([fu_replay], 5)
     (tf,) = timer.run([fu_replay], steps)
-    tfm = statistics.mean(tf)
+    tfm = statistics.median(tf)
     fl = case.causal_flops()
     ach = fl / tpm / 1e12
     store_bytes = 2 * 2 * kn.numel() * 2
@@ -468,8 +499,8 @@ def mixed_batch(device, timer, steps):
     timer.run([r1, r2], 5)
     t1, t2 = timer.run([r1, r2], steps)
     del r1, r2, _g1, _g2
-    return {"decode_rows": 64, "prompt_tokens": 4 * 512, "prefill_kernel_only_us": statistics.mean(t1) * 1e6,
-            "routed_us": statistics.mean(t2) * 1e6}
+    return {"decode_rows": 64, "prompt_tokens": 4 * 512, "prefill_kernel_only_us": statistics.median(t1) * 1e6,
+            "routed_us": statistics.median(t2) * 1e6}
 
 
 def block_size_sweep(device, pk, timer, steps):
@@ -486,12 +517,12 @@ def block_size_sweep(device, pk, timer, steps):
         rep, _g = capture(b.decode)
         timer.run([rep], 5)
         (t,) = timer.run([rep], steps)
-        tm = statistics.mean(t)
+        tm = statistics.median(t)
         res["decode"][str(B)] = {"decode_us": tm * 1e6, "kv_gbps": case.kv_bytes_read() / tm / 1e9,
                                  "frac": b.alg_bytes_decode() / tm / 1e9 / pk["hbm_gbs"]}
         del b, rep, _g
-    base = W.varlen_prefill(poison=False, keep_contiguous=False)
-    for B in (16, 64, 256):
+    base = get_case("varlen_prefill")
+    for B in (16, 32, 64, 128, 256):
         c = W.make_prefill_case(base.prompt_lens, base.cached_lens, 32, 8, 128, B, seed=2005, poison=False,
                                 keep_contiguous=False)
         kc, vc = c.k_cache.to(device), c.v_cache.to(device)
@@ -508,7 +539,7 @@ def block_size_sweep(device, pk, timer, steps):
         rep, _g = capture(pf)
         timer.run([rep], 5)
         (t,) = timer.run([rep], steps)
-        tm = statistics.mean(t)
+        tm = statistics.median(t)
         res["prefill"][str(B)] = {"prefill_us": tm * 1e6, "tflops": c.causal_flops() / tm / 1e12}
         del rep, _g
     torch.cuda.empty_cache()
@@ -527,55 +558,115 @@ def local_gpu_index(device):
 
 # ------------------------------------------------------------ CPU oracle --
 
-def oracle_decode_sample(case, n_seq, rng):
-    """Oracle store + decode of n_seq randomly chosen sequences (all q-heads); returns seconds."""
-    import oracle
-    seqs = rng.choice(case.batch, size=n_seq, replace=False)
-    t0 = time.perf_counter()
-    oracle.store(case.k_new, case.v_new, case.slot_mapping, case.k_cache, case.v_cache)
-    si = np.repeat(seqs, case.num_q_heads)
-    hi = np.tile(np.arange(case.num_q_heads), n_seq)
-    oracle.decode(case.q, case.k_cache, case.v_cache, case.block_table, case.context_lens, case.softmax_scale,
-                  seq_idx=si, head_idx=hi)
-    return time.perf_counter() - t0
+def _median_s(fn, reps=3):
+    """Wall-clock median of `reps` calls of fn (seconds)."""
+    ts = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        fn()
+        ts.append(time.perf_counter() - t0)
+    return statistics.median(ts)
 
 
-def cpu_baseline(case, budget_s=10.0):
+def oracle_store_s(case, reps=3):
+    """Wall-clock median of the oracle's row scatter of the step's new K/V rows, written in place into a
+    copy of the cache made once outside the timing (the rows it writes are the same every call)."""
     import oracle
-    rng = np.random.default_rng(0)
-    t1 = oracle_decode_sample(case, 8, rng)
-    reps, total, toks = 0, 0.0, 0
-    while total < budget_s and reps < 1000:
-        total += oracle_decode_sample(case, 8, rng)
-        toks += 8
-        reps += 1
-    return {"value": toks / total, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{reps} x (oracle store of all 64 rows + fp64 decode of 8 random sequences x 16 heads) "
-                      f"of the {PRIMARY} workload, {total:.1f} s; first call {t1:.2f} s excluded"}
+    kc, vc = case.k_cache.clone(), case.v_cache.clone()
+    return _median_s(lambda: oracle.store_inplace(case.k_new, case.v_new, case.slot_mapping, kc, vc), reps)
+
+
+def oracle_decode_s(case, seqs=None, reps=3):
+    """Wall-clock median of the oracle's decode of the given sequences (every q-head; all when None),
+    on the cache after the step's store (done once, outside the timing)."""
+    import oracle
+    kc, vc = case.k_cache.clone(), case.v_cache.clone()
+    oracle.store_inplace(case.k_new, case.v_new, case.slot_mapping, kc, vc)
+    if seqs is None:
+        call = lambda: oracle.decode(case.q, kc, vc, case.block_table, case.context_lens, case.softmax_scale)
+    else:
+        si = np.repeat(np.asarray(seqs), case.num_q_heads)
+        hi = np.tile(np.arange(case.num_q_heads), len(seqs))
+        call = lambda: oracle.decode(case.q, kc, vc, case.block_table, case.context_lens, case.softmax_scale,
+                                     seq_idx=si, head_idx=hi)
+    return _median_s(call, reps)
+
+
+def cpu_baseline(names, rows_frac_prefill=1.0 / 8):
+    """The fp64 CPU oracle as it stands, timed per workload and per call (store, decode, prefill) on this
+    host's cores: wall-clock median of 3 calls each.  Every decode call covers the whole batch; the
+    prefill is timed on a random 1/8 of its (token, head) rows and extrapolated to all of them (its cost
+    per row is what the row's key count makes it, and the sample is uniform over rows)."""
+    import oracle
+    res = {}
+    case = get_case(PRIMARY)
+    st, dec = oracle_store_s(case), oracle_decode_s(case)
+    res[PRIMARY] = {"store_s": st, "decode_s": dec, "tokens_per_s": case.batch / (st + dec),
+                    "kv_gbps": case.kv_bytes_read() / dec / 1e9, "sample": "whole batch"}
+    for name in [n for n in ("long_context_decode", "prefix_sharing_decode") if n in names]:
+        case = get_case(name)
+        st, dec = oracle_store_s(case), oracle_decode_s(case)
+        res[name] = {"store_s": st, "decode_s": dec, "tokens_per_s": case.batch / dec,
+                     "kv_gbps": case.kv_bytes_read() / dec / 1e9, "sample": "whole batch"}
+    if "varlen_prefill" in names:
+        case = get_case("varlen_prefill")
+        st = oracle_store_s(case)
+        kc, vc = case.k_cache.clone(), case.v_cache.clone()
+        oracle.store_inplace(case.k_new, case.v_new, case.slot_mapping, kc, vc)
+        rng = np.random.default_rng(0)
+        nrows = case.total_q * case.num_q_heads
+        pick = rng.choice(nrows, size=max(1, int(nrows * rows_frac_prefill)), replace=False)
+        ti, hi = pick // case.num_q_heads, pick % case.num_q_heads
+        t = _median_s(lambda: oracle.prefill(case.q, kc, vc, case.cu_seqlens_q, case.cu_seqlens_k,
+                                             case.block_table, case.softmax_scale, tok_idx=ti, head_idx=hi))
+        full = t * nrows / len(pick)
+        res["varlen_prefill"] = {"store_s": st, "store_rows": int(case.total_q),
+                                 "prefill_s_sample": t, "prefill_s_extrapolated": full,
+                                 "tflops": case.causal_flops() / full / 1e12,
+                                 "sample": f"{len(pick)} of {nrows} (token, head) rows, uniformly at random; "
+                                           f"time x {nrows / len(pick):.2f}"}
+    p = res[PRIMARY]
+    return {"value": p["tokens_per_s"], "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"{PRIMARY}: oracle store of the 64 new rows (in place) + fp64 decode of all 64 "
+                       f"sequences x 16 q-heads, wall-clock median of 3; per_config: every other workload, "
+                       f"median of 3 per call"),
+            "per_config": res}
 
 
 def run_reference(args, world, rank):
-    """The reference arm: the CPU oracle as it stands, a bounded sample per step (rank 0 only)."""
+    """The reference arm: the CPU oracle as it stands, a bounded sample per step (rank 0 only): the
+    store of the step's 64 new rows (in place) and the fp64 decode of a random subset of sequences."""
     if rank != 0:
         return
     import oracle
-    from paged_kv_cache_325_b200 import workloads as W
-    case = W.WORKLOADS[PRIMARY](poison=False, keep_contiguous=False)
+    case = get_case(PRIMARY)
+    kc, vc = case.k_cache.clone(), case.v_cache.clone()
     rng = np.random.default_rng(0)
-    t1 = oracle_decode_sample(case, 1, rng)
+
+    def step(n_seq):
+        seqs = rng.choice(case.batch, size=n_seq, replace=False)
+        si = np.repeat(seqs, case.num_q_heads)
+        hi = np.tile(np.arange(case.num_q_heads), n_seq)
+        t0 = time.perf_counter()
+        oracle.store_inplace(case.k_new, case.v_new, case.slot_mapping, kc, vc)
+        oracle.decode(case.q, kc, vc, case.block_table, case.context_lens, case.softmax_scale,
+                      seq_idx=si, head_idx=hi)
+        return time.perf_counter() - t0
+
+    t1 = step(1)
     per_step_budget = 90.0 / max(1, args.steps + args.warmup)
     n_seq = int(max(1, min(case.batch, per_step_budget / max(t1, 1e-3))))
     for _ in range(args.warmup):
-        oracle_decode_sample(case, n_seq, rng)
-    ts = [oracle_decode_sample(case, n_seq, rng) for _ in range(args.steps)]
+        step(n_seq)
+    ts = [step(n_seq) for _ in range(args.steps)]
     value = n_seq * args.steps / sum(ts)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(ts) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": PRIMARY_DESC, "parallelism": "replicas", "l2": "n/a (CPU)"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-                             "sample": f"per step: oracle store of 64 rows + fp64 decode of {n_seq} random "
-                                       f"sequences x 16 heads of the {PRIMARY} workload"},
+                             "sample": f"per step: oracle store of the 64 new rows (in place) + fp64 decode of "
+                                       f"{n_seq} random sequences x 16 heads of the {PRIMARY} workload"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -588,7 +679,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
-    ap.add_argument("--secondary", default="long_context_decode,prefix_sharing_decode,varlen_prefill,mixed_batch",
+    ap.add_argument("--secondary",
+                    default="long_context_decode,prefix_sharing_decode,varlen_prefill,mixed_batch,block_size_sweep",
                     help="comma list of extra workloads to time at N=1 ('none' for none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
@@ -618,7 +710,7 @@ def main(argv=None):
             secondary = bench_secondary(args, device, pk, names)
         cpu = None
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            cpu = cpu_baseline(case)
+            cpu = cpu_baseline(names)
     finally:
         if world > 1:
             import torch.distributed as dist

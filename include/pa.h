@@ -173,7 +173,10 @@ PA_API pa_status pa_decode(void *out, const void *q, const void *k_cache, const 
  * + (context_lens[s]-1) % block_size.  A different slot is still written, but
  * the decode does not see the new row there; checked mode reports it as
  * PA_DEVERR_SLOT, as it does a slot >= num_blocks * block_size (not written).
- * A row of a sequence whose context length is invalid is not stored.
+ * A row of a sequence whose context length is rejected (below 1, above
+ * max_context_len or past its block_table row; checked mode reports
+ * PA_DEVERR_CONTEXT_LEN) is still stored, as pa_store_kv would store it; only
+ * that sequence's decode is skipped and its output rows are left untouched.
  *
  *   k, v          [batch, num_kv_heads, head_dim] bf16, row s at element
  *                 s * k_row_stride (v_row_stride); the rows must be 16-byte
@@ -252,9 +255,11 @@ PA_API pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k
  *
  * Arguments are those of pa_decode without the workspace.  Sizes whose split
  * scratch (pa_decode_workspace_size) exceeds the array are rejected with
- * PA_ERR_WORKSPACE before anything is enqueued.  The first call on a device
- * looks up the array's device address (cudaGetSymbolAddress, that device
- * current) and caches it; make that first call before any stream capture.
+ * PA_ERR_WORKSPACE before anything is enqueued.  Every call looks up the
+ * array's address in the current device's context (cudaGetSymbolAddress) and
+ * keeps nothing, so the call stays correct after the context is torn down and
+ * created again (cudaDeviceReset); the first call on a device may load the
+ * library's device code, so make it before any stream capture.
  * Every call on a device shares the one array and it keeps the last call's
  * contents; nothing in it has to start at zero (each call writes every
  * partial it reads).  Calls whose kernels overlap on the GPU -- on different

@@ -87,6 +87,20 @@ class Oracle:
         to_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).reshape(k_cache.shape)
         return to_t(kc), to_t(vc)
 
+    def store_inplace(self, k, v, slot_mapping, k_cache, v_cache):
+        """The same row copy as store(), written into k_cache / v_cache themselves (contiguous CPU bf16
+        tensors) instead of into fresh copies of them, so that timing it measures the scatter alone."""
+        assert k_cache.is_contiguous() and v_cache.is_contiguous()
+        kb, vb = _bits(k), _bits(v)
+        kc = k_cache.view(torch.int16).numpy().view(np.uint16)
+        vc = v_cache.view(torch.int16).numpy().view(np.uint16)
+        sm = _i32(slot_mapping)
+        nb, B, Hkv, D = k_cache.shape
+        rc = self.lib.oracle_store(_p(kb, _U16P), _p(vb, _U16P), Hkv * D, Hkv * D, _p(sm, _I32P), len(sm),
+                                   _p(kc, _U16P), _p(vc, _U16P), nb * B, Hkv, D)
+        if rc != 0:
+            raise ValueError("oracle_store: slot out of range")
+
     def decode(self, q, k_cache, v_cache, block_table, context_lens, softmax_scale, seq_idx=None,
                head_idx=None):
         """fp64 decode attention.  Returns [batch, Hq, D], or [len(seq_idx), D] for sampled pairs."""
@@ -153,6 +167,10 @@ def num_threads() -> int:
 
 def store(*a, **kw):
     return default().store(*a, **kw)
+
+
+def store_inplace(*a, **kw):
+    return default().store_inplace(*a, **kw)
 
 
 def decode(*a, **kw):

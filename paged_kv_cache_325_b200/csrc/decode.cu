@@ -205,6 +205,31 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         }
     }
     __syncthreads();
+    if (a.new_slots) {
+        // fused store: a sequence whose context length is rejected gets no item, so no decode warp stores
+        // its new row; store it here (one warp per such sequence), as pa_store_kv would
+        const int lane = tid & 31;
+        const int chunks = a.num_kv_heads * a.head_dim / 8;    // 16-byte pieces of one K (or V) row
+        for (int s = tid >> 5; s < a.batch; s += kPlanThreads / 32) {
+            if (dec_tiles(a, s, false) > 0) continue;
+            const int32_t sl = __ldg(a.new_slots + s);
+            if (sl < 0) continue;
+            if ((int64_t)sl >= a.num_slots) {
+                if (lane == 0) report(a.dev_error, PA_DEVERR_SLOT);
+                continue;
+            }
+            const uint4 *ks = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.k_new) +
+                                                              (int64_t)s * a.kn_stride);
+            const uint4 *vs = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.v_new) +
+                                                              (int64_t)s * a.vn_stride);
+            uint4 *kd = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.k_cache) + (int64_t)sl * chunks * 8);
+            uint4 *vd = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.v_cache) + (int64_t)sl * chunks * 8);
+            for (int c = lane; c < chunks; c += 32) {
+                kd[c] = __ldg(ks + c);
+                vd[c] = __ldg(vs + c);
+            }
+        }
+    }
     int4 *items = reinterpret_cast<int4 *>(reinterpret_cast<char *>(a.plan_ws) + kPlanHdrBytes);
     const int64_t npairs = (int64_t)a.batch * a.num_kv_heads;
     for (int64_t pr = tid; pr < npairs; pr += kPlanThreads) {

@@ -9,11 +9,12 @@
 // The array is a file-scope __device__ variable, so every GPU that loads the
 // library holds kNoAllocScratchBytes of it until the process exits.  Host code
 // must not pass the variable's name to a kernel (on the host that name is a
-// stand-in, not a device address); the device address is looked up once per
-// device with cudaGetSymbolAddress, with that device current, and cached.
+// stand-in, not a device address).  Every call asks the runtime for the
+// array's address on the current device (cudaGetSymbolAddress, a table lookup
+// once the module is loaded) instead of keeping it: after a cudaDeviceReset,
+// or any other teardown of the context, the module is loaded again and the
+// array may sit elsewhere, so a kept address could point at freed memory.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "pa.h"
 #include "pa_internal.h"
@@ -21,36 +22,18 @@
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB per device
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
-std::mutex g_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_decode_scratch on the current device (looked up on first use).
+// Device address of g_decode_scratch in the current device's context.
 pa_status scratch_for_current_device(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) {
-        pa::set_last_error(PA_ERR_CUDA, "pa_decode_noalloc: cudaGetDevice failed");
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess || !p) {
+        pa::set_last_error(PA_ERR_CUDA, "pa_decode_noalloc: cudaGetSymbolAddress of the static scratch failed");
         return PA_ERR_CUDA;
     }
-    if (dev < 0 || dev >= kMaxDevices) {
-        pa::set_last_error(PA_ERR_UNSUPPORTED, "pa_decode_noalloc: device index out of range");
-        return PA_ERR_UNSUPPORTED;
-    }
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_decode_scratch);
-        if (e != cudaSuccess || !p) {
-            pa::set_last_error(PA_ERR_CUDA, "pa_decode_noalloc: cudaGetSymbolAddress of the static scratch failed");
-            return PA_ERR_CUDA;
-        }
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return PA_OK;
 }
 

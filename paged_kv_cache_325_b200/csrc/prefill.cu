@@ -802,7 +802,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st16(lane_base + col_s(x) + kc * 16, w);
                 }
                 l = l * corr + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-                if (rescale && j > 0) {
+                // The decision is per row, but tcgen05.ld / st are warp-wide (.sync.aligned): the whole warp
+                // takes the branch when any of its rows rescales, and the other rows multiply by corr = 1.
+                if (__any_sync(0xffffffffu, rescale && j > 0)) {
                     // O_X is stable: PV_X(j-1) completed before S_X(j), which was issued after it
 #pragma unroll
                     for (int q = 0; q < D / 32; ++q) {

@@ -272,15 +272,27 @@ def make_decode_case(context_lens, num_q_heads, num_kv_heads, head_dim, block_si
                       k_seq=k_seq, v_seq=v_seq, shared_prefix_blocks=P)
 
 
+def _ramp_keys(ks: torch.Tensor, key_growth: float) -> torch.Tensor:
+    """Scale the K row at position p by 1 + key_growth * p / 128 (rounded back to bf16), so that the
+    attention scores of later keys spread ever wider: the running maximum of a query's scores keeps
+    rising along the sequence.  key_growth = 0 returns the rows untouched."""
+    if not key_growth:
+        return ks
+    ramp = 1.0 + key_growth * torch.arange(ks.shape[0], dtype=torch.float32) / 128.0
+    return (ks.float() * ramp[:, None, None]).to(torch.bfloat16)
+
+
 def make_prefill_case(prompt_lens, cached_lens, num_q_heads, num_kv_heads, head_dim, block_size,
                       num_blocks=None, seed=0, poison=True, keep_contiguous=True, causal=True,
-                      name="prefill", softmax_scale=None) -> PrefillCase:
+                      name="prefill", softmax_scale=None, key_growth=0.0) -> PrefillCase:
     """Build one varlen prefill step.
 
     Sequence s has prompt_lens[s] tokens; its first cached_lens[s] tokens (a
     whole number of blocks) already sit in the cache from a prefix-cache hit,
     the remaining n_new = prompt_len - cached_len tokens are stored this step
-    and are the queries.
+    and are the queries.  ``key_growth`` > 0 scales the K row at position p
+    by 1 + key_growth * p / 128 (see ``_ramp_keys``); it draws no extra random
+    numbers, so the other values are those of the same seed without it.
     """
     rng = np.random.Generator(np.random.PCG64(seed))
     L = np.asarray(prompt_lens, dtype=np.int32)
@@ -316,7 +328,7 @@ def make_prefill_case(prompt_lens, cached_lens, num_q_heads, num_kv_heads, head_
     k_seq, v_seq = ([], []) if keep_contiguous else (None, None)
     for s in range(batch):
         n = int(L[s])
-        ks = _normal_bf16(rng, (n, Hkv, D))
+        ks = _ramp_keys(_normal_bf16(rng, (n, Hkv, D)), key_growth)
         vs = _normal_bf16(rng, (n, Hkv, D))
         cs = int(c[s])
         _scatter_tokens(k_cache, block_table[s], ks[:cs], 0, B)

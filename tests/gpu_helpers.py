@@ -1,5 +1,7 @@
 """Shared helpers of the GPU parity tests: run a workload through the C ABI and
 through the CPU oracle on the same seeded bytes, and compare."""
+import functools
+
 import numpy as np
 import torch
 
@@ -103,3 +105,12 @@ def oracle_prefill(case, tok_idx=None, head_idx=None, causal=None):
     return oracle.prefill(case.q, kc, vc, case.cu_seqlens_q, case.cu_seqlens_k, case.block_table,
                           case.softmax_scale, causal=case.causal if causal is None else causal,
                           tok_idx=tok_idx, head_idx=head_idx)
+
+
+@functools.lru_cache(maxsize=1)
+def varlen_prefill_reference():
+    """The full-size varlen prefill workload (poisoned parity form) and the oracle's result for every
+    (new token, q-head) row; computed once per test session (about 10 s of fp64 on 16 threads)."""
+    from paged_kv_cache_325_b200 import workloads as W
+    case = W.varlen_prefill()
+    return case, oracle_prefill(case)

@@ -119,6 +119,29 @@ def test_store_decode_checked_mode(cuda_lib):
     assert torch.equal(g.v_cache.cpu().view(torch.int16), vc.view(torch.int16))
 
 
+def test_store_decode_stores_rows_of_rejected_sequences(cuda_lib):
+    """A sequence whose context length is rejected (0, or past max_context_len) gets no decode, but its
+    new row is still stored, as pa_store_kv then pa_decode would leave the cache; the other sequences'
+    outputs are unaffected and the rejected sequences' output rows are left as they were."""
+    case = W.make_decode_case([40, 300, 129, 77], 8, 2, 128, 16, seed=1707, poison=False)
+    ctx = case.context_lens.copy()
+    ctx[1] = 0                              # invalid: below 1
+    ctx[3] = case.max_context_len + 50      # invalid: past max_context_len
+    g = DecodeOnGpu(case)
+    g.context_lens = i32(ctx, g.dev)
+    err = torch.zeros(1, dtype=torch.int32, device=g.dev)
+    out = torch.full_like(g.q, 7.0)
+    _fused(g, dev_error=err, out=out)
+    torch.cuda.synchronize()
+    assert int(err.item()) & pa.PA_DEVERR_CONTEXT_LEN
+    _cache_equals_oracle_store(g, case)
+    ref = oracle_decode(case)
+    for s in (0, 2):
+        assert_close(out[s], ref[s], what=f"valid sequence {s}")
+    for s in (1, 3):
+        assert bool((out[s] == 7.0).all()), f"output of rejected sequence {s} was written"
+
+
 def test_store_decode_rejects_unaligned_rows(cuda_lib):
     case = W.tiny_decode()
     g = DecodeOnGpu(case)

@@ -5,7 +5,8 @@ KV pool).  Its split scratch is a fixed array inside the library.
 Calls the new entry point through the C ABI (ctypes on libpagedattn.so) and
 compares its output with pa_decode's on the same inputs, within the parity
 tolerance, on two calls in a row with different inputs (the shared scratch
-keeps the first call's contents when the second runs).  This file is collected
+keeps the first call's contents when the second runs), and both with the fp64
+oracle.  This file is collected
 last so that a stop-at-first-failure run has executed every other test first.
 """
 import ctypes
@@ -16,7 +17,7 @@ import torch
 
 import paged_kv_cache_325_b200 as pa
 from paged_kv_cache_325_b200 import workloads as W
-from gpu_helpers import MAX_ABS, MEAN_ABS, DecodeOnGpu
+from gpu_helpers import MAX_ABS, MEAN_ABS, DecodeOnGpu, assert_close, oracle_decode
 
 pytestmark = pytest.mark.gpu
 
@@ -55,6 +56,7 @@ def test_noalloc_matches_pa_decode_on_two_calls_in_a_row(cuda_lib):
         assert np.isfinite(a).all()
         err = np.abs(a - b)
         assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (case.name, err.max(), err.mean())
+        assert_close(got, oracle_decode(case), what=f"noalloc {case.name} vs oracle")
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_lib):

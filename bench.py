@@ -325,7 +325,7 @@ def bench_primary(args, world, rank, device, pk):
         st_replay, _g1 = capture(b.store)
         dec_replay, _g2 = capture(b.decode)
         timer.run([st_replay, dec_replay], 5)
-        steps2 = max(SECONDARY_STEPS, min(args.steps, 500))
+        steps2 = max(args.secondary_steps, min(args.steps, 500))
         t_store, t_dec = timer.run([st_replay, dec_replay], steps2)
         res["separate_launches"] = {"store_us": statistics.median(t_store) * 1e6,
                                     "decode_us": statistics.median(t_dec) * 1e6,
@@ -370,7 +370,7 @@ def bench_secondary(args, device, pk, names):
     from paged_kv_cache_325_b200 import workloads as W
     timer = Timer(device)
     out = {}
-    steps = SECONDARY_STEPS
+    steps = args.secondary_steps
     for name in [n for n in names if n in ("long_context_decode", "prefix_sharing_decode")]:
         case = get_case(name)
         b = DecodeBench(case, device)
@@ -603,6 +603,10 @@ def cpu_baseline(names, rows_frac_prefill=1.0 / 8):
     st, dec = oracle_store_s(case), oracle_decode_s(case)
     res[PRIMARY] = {"store_s": st, "decode_s": dec, "tokens_per_s": case.batch / (st + dec),
                     "kv_gbps": case.kv_bytes_read() / dec / 1e9, "sample": "whole batch"}
+    case = get_case("tiny_decode")
+    st, dec = oracle_store_s(case), oracle_decode_s(case)
+    res["tiny_decode"] = {"store_s": st, "decode_s": dec, "tokens_per_s": case.batch / (st + dec),
+                          "sample": "whole batch"}
     for name in [n for n in ("long_context_decode", "prefix_sharing_decode") if n in names]:
         case = get_case(name)
         st, dec = oracle_store_s(case), oracle_decode_s(case)
@@ -683,6 +687,10 @@ def main(argv=None):
                     default="long_context_decode,prefix_sharing_decode,varlen_prefill,mixed_batch,block_size_sweep",
                     help="comma list of extra workloads to time at N=1 ('none' for none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--secondary-steps", type=int, default=SECONDARY_STEPS,
+                    help="timed runs per secondary measurement (median reported)")
+    ap.add_argument("--secondary-only", action="store_true",
+                    help="time only the --secondary workloads (no primary line; for profiling one workload)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -702,6 +710,13 @@ def main(argv=None):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     pk, peak_src = peaks()
+    if args.secondary_only:
+        if world != 1:
+            raise SystemExit("--secondary-only runs on one GPU")
+        names = [n for n in args.secondary.split(",") if n and n != "none"]
+        print(json.dumps({"secondary_only": True, "peak_source": peak_src,
+                          "workloads": bench_secondary(args, device, pk, names)}), flush=True)
+        return 0
     try:
         case, res = bench_primary(args, world, rank, device, pk)
         secondary = None

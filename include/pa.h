@@ -383,6 +383,19 @@ PA_API pa_status pa_store_kv_prefill_varlen(const void *k, const void *v, int64_
  */
 PA_API pa_status pa_selftest_bounded_wait(int32_t *dev_error, int64_t max_polls, void *stream);
 
+/*
+ * pa_selftest_exp2 -- evaluates, for each x[i] (device float array of n
+ * values), the two ways the prefill softmax computes 2^x: y_poly[i] from the
+ * library's own polynomial on the FMA pipe (round-to-nearest range reduction
+ * and a degree-3 fit of 2^f on [-1/2, 1/2], relative error below 1e-4; inputs
+ * below -125 give 2^-125) and y_sfu[i] from the special-function unit's
+ * ex2.approx.  All three arrays are caller-owned device memory.  Used by the
+ * tests to hold the polynomial to its error bound; has no counterpart in the
+ * attention method itself.  Errors: PA_ERR_INVALID_ARG for n < 0 or NULL /
+ * misaligned arrays.
+ */
+PA_API pa_status pa_selftest_exp2(const float *x, float *y_poly, float *y_sfu, int32_t n, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -9,5 +9,5 @@ from ._binding import (  # noqa: F401
     PA_OK, PagedAttnError, alloc_decode_workspace, alloc_mixed_workspace, alloc_prefill_workspace, alloc_shared_prefix_workspace, declared_symbols, load_library, pa_decode, pa_decode_noalloc, pa_decode_shared_prefix, pa_decode_shared_prefix_workspace_size, pa_decode_split,
     pa_decode_split_workspace_size, pa_decode_workspace_size, pa_prefill_varlen, pa_prefill_varlen_mixed,
     pa_prefill_varlen_mixed_workspace_size, pa_prefill_workspace_size,
-    pa_selftest_bounded_wait, pa_status_string, pa_store_kv, pa_store_kv_decode, pa_store_kv_prefill_varlen, pa_version,
+    pa_selftest_bounded_wait, pa_selftest_exp2, pa_status_string, pa_store_kv, pa_store_kv_decode, pa_store_kv_prefill_varlen, pa_version,
 )

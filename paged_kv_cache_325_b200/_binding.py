@@ -37,7 +37,8 @@ __all__ = ["PagedAttnError", "load_library", "declared_symbols", "pa_store_kv", 
            "pa_prefill_varlen_mixed_workspace_size", "alloc_mixed_workspace",
            "pa_decode_workspace_size", "pa_decode_split_workspace_size", "pa_decode_noalloc",
            "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size", "alloc_shared_prefix_workspace", "pa_prefill_varlen",
-           "pa_prefill_workspace_size", "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
+           "pa_prefill_workspace_size", "pa_selftest_bounded_wait", "pa_selftest_exp2", "pa_status_string",
+           "pa_version",
            "alloc_decode_workspace", "alloc_prefill_workspace"]
 
 
@@ -83,6 +84,7 @@ _SIGS = {
                                                _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_f32, _c_p,
                                                _c_sz, _c_p, _c_p]),
     "pa_selftest_bounded_wait": (ctypes.c_int, [_c_p, _c_i64, _c_p]),
+    "pa_selftest_exp2": (ctypes.c_int, [_c_p, _c_p, _c_p, _c_i32, _c_p]),
 }
 
 
@@ -417,3 +419,12 @@ def pa_selftest_bounded_wait(dev_error, max_polls, stream=None):
     import torch
     _need(dev_error, "dev_error", torch.int32)
     _check(load_library().pa_selftest_bounded_wait(_ptr(dev_error), int(max_polls), _stream(dev_error, stream)))
+
+
+def pa_selftest_exp2(x, stream=None):
+    """Evaluate the prefill softmax's two exponentials on a float32 CUDA tensor x: returns (y_poly, y_sfu)."""
+    import torch
+    _need(x, "x", dtype=torch.float32)
+    y_poly, y_sfu = torch.empty_like(x), torch.empty_like(x)
+    _check(load_library().pa_selftest_exp2(_ptr(x), _ptr(y_poly), _ptr(y_sfu), x.numel(), _stream(x, stream)))
+    return y_poly, y_sfu

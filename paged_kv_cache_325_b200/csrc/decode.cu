@@ -94,6 +94,7 @@ struct DecPlanHdr {
 constexpr int kPlanHdrBytes = 256;
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBuckets = 1024;          // item lengths (tiles) for the longest-first order; longer share the last
+constexpr int kPlanCache = 2048;            // sequences whose length the planning kernel keeps in shared memory
 
 // Context length of sequence s: context_lens[s]; in the varlen mode (the decode rows of a mixed batch) the
 // key count of a sequence with exactly one new token, and -1 for any other sequence (not this call's work).
@@ -130,6 +131,8 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the decode kernel may start its set-up
     __shared__ unsigned long long s_total;
     __shared__ int s_off[kPlanBuckets];
+    // tiles and context length of the first kPlanCache sequences, read once from global memory
+    __shared__ int s_tiles[kPlanCache], s_ctx[kPlanCache];
     const int tid = threadIdx.x;
     if (tid == 0) s_total = 0;
     for (int b = tid; b < kPlanBuckets; b += kPlanThreads) s_off[b] = 0;
@@ -137,7 +140,12 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     // total work in tiles; checked mode: context lengths and the shared blocks
     unsigned long long part = 0;
     for (int s = tid; s < a.batch; s += kPlanThreads) {
-        part += (unsigned long long)dec_tiles(a, s, true) * a.num_kv_heads;
+        const int tiles = dec_tiles(a, s, true);
+        if (s < kPlanCache) {
+            s_tiles[s] = tiles;
+            s_ctx[s] = dec_ctx(a, s);
+        }
+        part += (unsigned long long)tiles * a.num_kv_heads;
         if (a.dev_error && a.shared_blocks > 0)
             for (int b = 0; b < a.shared_blocks; ++b)
                 if (__ldg(a.block_table + (int64_t)s * a.bt_stride + b) != __ldg(a.block_table + b))
@@ -146,8 +154,9 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
     if ((tid & 31) == 0) atomicAdd(&s_total, part);
     __syncthreads();
-    // split rule: pairs up to the average per-CTA load stay whole; longer ones are cut into pieces of an
-    // eighth of it (never finer than the host's chunk, which sized the partial slots)
+    // split rule: pairs up to the average per-CTA load stay whole; longer ones are cut into pieces of a
+    // sixteenth of it (never finer than the host's chunk, which sized the partial slots), so that the last
+    // pieces handed out -- and with them the spread of the CTAs' finishing times -- stay short
     int whole, chunk;
     const int host_chunk = a.plan.chunk / kTile;
     if (a.plan.fixed) {
@@ -157,13 +166,13 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         const unsigned long long avg = (s_total + num_ctas - 1) / (unsigned long long)num_ctas;
         whole = (int)min(avg, 1ull << 30);
         if (whole < 4) whole = 4;
-        chunk = (int)min((avg + 7) / 8, 1ull << 30);
+        chunk = (int)min((avg + 15) / 16, 1ull << 30);
         if (chunk < host_chunk) chunk = host_chunk;
     }
     // longest-first order: count items per length bucket, then exclusive offsets from the longest bucket
     auto bucket = [](int tiles) { return min(tiles, kPlanBuckets - 1); };
     for (int s = tid; s < a.batch; s += kPlanThreads) {
-        const int tiles = dec_tiles(a, s, false);
+        const int tiles = s < kPlanCache ? s_tiles[s] : dec_tiles(a, s, false);
         const int n = dec_nsplit(tiles, whole, chunk);
         if (n == 0) continue;
         if (n == 1) {
@@ -198,7 +207,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         s_off[b] = inc - v + (w > 0 ? s_warp[w - 1] : 0);
         if (tid == kPlanThreads - 1) {
             DecPlanHdr *h = reinterpret_cast<DecPlanHdr *>(a.plan_ws);
-            h->counter = 0;
+            h->counter = num_ctas;          // item c < num_ctas is CTA c's first item (taken without the counter)
             h->n_items = s_warp[kPlanThreads / 32 - 1];
             h->whole = whole;
             h->chunk = chunk;
@@ -234,10 +243,10 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     const int64_t npairs = (int64_t)a.batch * a.num_kv_heads;
     for (int64_t pr = tid; pr < npairs; pr += kPlanThreads) {
         const int s = (int)(pr / a.num_kv_heads), kvh = (int)(pr % a.num_kv_heads);
-        const int tiles = dec_tiles(a, s, false);
+        const int tiles = s < kPlanCache ? s_tiles[s] : dec_tiles(a, s, false);
         const int n = dec_nsplit(tiles, whole, chunk);
         if (n == 0) continue;
-        const int ctx = dec_ctx(a, s);
+        const int ctx = s < kPlanCache ? s_ctx[s] : dec_ctx(a, s);
         if (n == 1) {
             items[atomicAdd(&s_off[bucket(tiles)], 1)] = make_int4(s, kvh, a.t_offset, ctx);
             continue;
@@ -286,6 +295,9 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     int4 *desc = reinterpret_cast<int4 *>(smem + C::kBarOff + 192);   // [2]: the item of each Q slot
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the combine kernel (launched next, as this grid's programmatic dependent) may be scheduled now: its CTAs
+    // only wait (griddepcontrol.wait) for this grid to finish, in resources this one leaves free
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t ring = smem_u32(smem);
     const uint32_t qsm = ring + C::kQOff;
     const uint32_t qslot = (uint32_t)(G * D * 2);
@@ -320,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int4 *items = reinterpret_cast<const int4 *>(reinterpret_cast<const char *>(a.plan_ws) + kPlanHdrBytes);
             const int n_items = __ldcg(&hdr->n_items);
             const int4 kEnd = make_int4(-1, 0, 0, 0);
-            int idx = atomicAdd(&hdr->counter, 1);
+            int idx = blockIdx.x;               // the first item is this CTA's own; the rest come from the counter
             int4 d = idx < n_items ? __ldcg(items + idx) : kEnd;
             while (ok) {
                 const int qs = nqi & 1;
@@ -646,49 +658,101 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-// Merge the per-split partials of one (sequence, q-head) by log-sum-exp.  D threads, one per output
-// element.  Every warp reads the log-sum-exps 32 at a time (one per lane) and reduces them with shuffles;
-// the partial rows are then read in unrolled batches, so a merge costs a few L2 round trips, not two per
-// split.
-template <int D>
-__global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
-    asm volatile("griddepcontrol.wait;" ::: "memory");   // partials of the split kernel are visible
+// Merge the per-split partials of one (sequence, q-head) by log-sum-exp.  kGroups x D threads: thread
+// (g, d) owns output element d for the partial slots g, g + kGroups, ...  The merge is a chain of dependent
+// reads, so it is kept short: the context length (an input of the call) is read before the wait for the
+// split kernel; after it, the planning header, the log-sum-exps and -- in the wide form, for the slot count
+// the host sized -- the first kPre partial elements of every thread are all requested at once, and the
+// slots past this pair's count are selected out afterwards.  The kGroups sums are added in shared memory.  A
+// pair that was not split returns at once (kGroups = 1 when no pair can have more than a few partials).
+constexpr int kLseCache = 1024;
+
+template <int D, int kGroups>
+__global__ void __launch_bounds__(D * kGroups) decode_combine_kernel(const DecodeArgs a) {
+    constexpr int kPre = kGroups > 1 ? 16 : 4;     // partial elements per thread requested with the header
     const int h = blockIdx.x % a.num_q_heads;
     const int s = blockIdx.x / a.num_q_heads;
     const int ctx = dec_ctx(a, s);              // -1: not this call's work
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // partials of the split kernel are visible
     if (ctx < 1 || ctx > a.max_context_len || (int64_t)ctx > (int64_t)a.bt_stride * a.block_size ||
         ctx < a.t_offset)
         return;
     // partials: part_base slots written before this launch (shared-prefix chunks), then the splits, cut as
     // the planning kernel cut them; a pair of one split and nothing else was written directly
     const DecPlanHdr *hdr = reinterpret_cast<const DecPlanHdr *>(a.plan_ws);
-    const int nsplit = dec_nsplit((ctx - a.t_offset + kTile - 1) / kTile, __ldcg(&hdr->whole), __ldcg(&hdr->chunk));
-    if (a.part_base == 0 && nsplit <= 1) return;
-    const int n = a.part_base + nsplit;
     const int64_t base = ((int64_t)s * a.num_q_heads + h) * a.part_slots;
-    const int d = threadIdx.x, lane = d & 31;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int g = tid / D, d = tid % D;
+    const int nmax = a.part_slots;              // slots of this pair: an upper bound of its partial count
     const float *lse = a.part_lse + base;
     const float *po = a.part_o + base * D + d;
+    const int whole = __ldcg(&hdr->whole), chunk = __ldcg(&hdr->chunk);
+    float l0 = tid < nmax ? __ldcg(lse + tid) : -INFINITY;
+    float pv[kPre];
+    if (kGroups > 1) {
+#pragma unroll
+        for (int i = 0; i < kPre; ++i) {
+            const int k = g + i * kGroups;
+            pv[i] = k < nmax ? __ldcg(po + (int64_t)k * D) : 0.f;
+        }
+    }
+    const int nsplit = dec_nsplit((ctx - a.t_offset + kTile - 1) / kTile, whole, chunk);
+    if (a.part_base == 0 && nsplit <= 1) return;
+    const int n = a.part_base + nsplit;
+    if (kGroups == 1) {
+#pragma unroll
+        for (int i = 0; i < kPre; ++i) pv[i] = i < n ? __ldcg(po + (int64_t)i * D) : 0.f;
+    }
+    constexpr int kWarps = D * kGroups / 32;
+    __shared__ float s_lse[kLseCache];
+    __shared__ float s_red[kWarps];
+    __shared__ float s_num[kGroups][D];
+    __shared__ float s_den[kGroups];
+    // 1. the largest log-sum-exp
+    float mx = -INFINITY;
+    for (int k = tid; k < n; k += D * kGroups) {
+        const float l = k == tid ? l0 : lse[k];
+        if (k < kLseCache) s_lse[k] = l;
+        mx = fmaxf(mx, l);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) s_red[wid] = mx;
+    __syncthreads();
     float mt = -INFINITY;
-    for (int k0 = 0; k0 < n; k0 += 32) {
-        float l = k0 + lane < n ? lse[k0 + lane] : -INFINITY;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) l = fmaxf(l, __shfl_xor_sync(0xffffffffu, l, o));
-        mt = fmaxf(mt, l);
+    for (int w = 0; w < kWarps; ++w) mt = fmaxf(mt, s_red[w]);
+    // 2. this thread's share of the weighted sum (slots past n are selected out, never multiplied)
+    float num = 0.f, den = 0.f;
+#pragma unroll
+    for (int i = 0; i < kPre; ++i) {
+        const int k = g + i * kGroups;
+        if (k < n) {
+            const float l = k < kLseCache ? s_lse[k] : lse[k];
+            const float w = l == -INFINITY ? 0.f : fast_exp2(l - mt);
+            den += w;
+            num += w * pv[i];
+        }
     }
-    float den_lane = 0.f, num = 0.f;
-    for (int k0 = 0; k0 < n; k0 += 32) {
-        const float l = k0 + lane < n ? lse[k0 + lane] : -INFINITY;
-        const float w = l == -INFINITY ? 0.f : fast_exp2(l - mt);
-        den_lane += w;
-        const int m = min(32, n - k0);
 #pragma unroll 8
-        for (int j = 0; j < m; ++j) num += __shfl_sync(0xffffffffu, w, j) * po[(int64_t)(k0 + j) * D];
+    for (int k = g + kPre * kGroups; k < n; k += kGroups) {
+        const float l = k < kLseCache ? s_lse[k] : lse[k];
+        const float w = l == -INFINITY ? 0.f : fast_exp2(l - mt);
+        den += w;
+        num += w * po[(int64_t)k * D];
     }
+    if (kGroups > 1) {
+        s_num[g][d] = num;
+        if (d == 0) s_den[g] = den;
+        __syncthreads();
+        if (g != 0) return;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den_lane += __shfl_xor_sync(0xffffffffu, den_lane, o);
-    static_cast<__nv_bfloat16 *>(a.out)[(dec_row(a, s) * a.num_q_heads + h) * D + d] =
-        __float2bfloat16_rn(num / den_lane);
+        for (int q = 1; q < kGroups; ++q) {
+            num += s_num[q][d];
+            den += s_den[q];
+        }
+    }
+    static_cast<__nv_bfloat16 *>(a.out)[(dec_row(a, s) * a.num_q_heads + h) * D + d] = __float2bfloat16_rn(num / den);
 }
 
 template <int D>
@@ -738,10 +802,16 @@ cudaError_t launch_decode_d(const DecodeArgs &a, const CUtensorMap &tm_k, const 
     e = cudaLaunchKernelEx(&cfg, kernel, tm_k, tm_v, a);
     if (e != cudaSuccess || (a.plan.max_splits == 1 && a.part_base == 0)) return e;
 
+    // a few partials per pair, or so many pairs that four threads per element would not fit the GPU at
+    // once (a large batch): one thread per element; many partials for few pairs (long contexts): four
+    // threads per element, each loading a quarter of them
+    const int64_t wide_threads = (int64_t)a.batch * a.num_q_heads * 4 * D;
+    const bool wide = a.part_base + a.plan.max_splits > 8 && wide_threads <= (int64_t)sms * 1024;
     cfg.gridDim = dim3((unsigned)(a.batch * a.num_q_heads));
-    cfg.blockDim = dim3(D);
+    cfg.blockDim = dim3(wide ? 4 * D : D);
     cfg.dynamicSmemBytes = 0;
-    return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, a);
+    return wide ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<D, 4>, a)
+                : cudaLaunchKernelEx(&cfg, decode_combine_kernel<D, 1>, a);
 }
 
 }  // namespace
@@ -755,9 +825,9 @@ DecodePlan plan_decode(int32_t batch, int32_t num_kv_heads, int32_t max_context_
         chunk = ((int64_t)max_context_len + num_splits - 1) / num_splits;
         chunk = (chunk + kTile - 1) / kTile * kTile;
     } else {
-        // aim at about eight waves of two CTAs per SM over the whole batch, but
+        // aim at about sixteen waves of two CTAs per SM over the whole batch, but
         // never fewer than four tiles per CTA
-        const int64_t target = (int64_t)(num_sms > 0 ? num_sms : 148) * 2 * 8;
+        const int64_t target = (int64_t)(num_sms > 0 ? num_sms : 148) * 2 * 16;
         const int64_t pairs = (int64_t)batch * num_kv_heads;
         chunk = ((int64_t)max_context_len * pairs + target - 1) / target;
         chunk = (chunk + kTile - 1) / kTile * kTile;

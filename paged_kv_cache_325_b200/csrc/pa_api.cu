@@ -714,4 +714,14 @@ pa_status pa_selftest_bounded_wait(int32_t *dev_error, int64_t max_polls, void *
     return ok();
 }
 
+pa_status pa_selftest_exp2(const float *x, float *y_poly, float *y_sfu, int32_t n, void *stream) {
+    if (n < 0) return fail(PA_ERR_INVALID_ARG, "n < 0");
+    if (n == 0) return ok();
+    if (!x || !y_poly || !y_sfu || !aligned(x, 4) || !aligned(y_poly, 4) || !aligned(y_sfu, 4))
+        return fail(PA_ERR_INVALID_ARG, "x, y_poly and y_sfu must be float arrays in device memory");
+    cudaError_t e = pa::launch_selftest_exp2(x, y_poly, y_sfu, n, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+    return ok();
+}
+
 }  // extern "C"

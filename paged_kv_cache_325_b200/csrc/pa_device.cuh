@@ -15,8 +15,9 @@
 namespace pa {
 
 // Every bounded wait gives up after this much wall-clock time (read from the
-// %globaltimer nanosecond clock), far beyond any legitimate wait here.
-constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
+// %globaltimer nanosecond clock), far beyond any legitimate wait here (the
+// kernels' waits are microseconds; a whole launch takes well under a millisecond).
+constexpr uint64_t kWaitTimeoutNs = 1000000000ull;
 
 PA_DEVICE uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -83,14 +84,23 @@ PA_DEVICE uint64_t global_timer_ns() {
 
 // Wait for the phase with the given parity to complete.  Returns false (and
 // reports PA_DEVERR_TIMEOUT) if it did not complete within kWaitTimeoutNs or
-// within `max_polls` polls, whichever comes first.
-PA_DEVICE bool mbar_wait(uint32_t bar, uint32_t parity, int32_t *dev_error, uint32_t max_polls = 0xffffffffu) {
+// within `max_polls` polls, whichever comes first.  With `abort` (a flag in
+// shared memory that every role of the CTA passes), a wait that gives up sets
+// the flag and every other wait of the CTA then gives up at its next check
+// instead of running into its own time limit: a CTA whose protocol broke
+// leaves after one time limit, not after one per remaining wait.
+PA_DEVICE bool mbar_wait(uint32_t bar, uint32_t parity, int32_t *dev_error, uint32_t max_polls = 0xffffffffu,
+                         volatile int32_t *abort = nullptr) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1; i < max_polls; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0 && global_timer_ns() - t0 > kWaitTimeoutNs) break;
+        if ((i & 63u) == 0) {
+            if (abort && *abort) return false;
+            if (global_timer_ns() - t0 > kWaitTimeoutNs) break;
+        }
     }
+    if (abort) *abort = 1;
     report(dev_error, PA_DEVERR_TIMEOUT);
     return false;
 }
@@ -163,6 +173,62 @@ PA_DEVICE float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic: one instruction for two lanes' worth of work).  The pair
+// lives in a 64-bit register; `lo` is the first element.
+PA_DEVICE uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+PA_DEVICE void f2_unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+PA_DEVICE uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {   // a * b + c, round to nearest, per element
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+PA_DEVICE uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// 2^x for a pair of fp32 on the FMA pipe, for the part of a softmax's exponentials that the special-function
+// unit (ex2, which runs at a fraction of the FMA rate) cannot take in time.  Written from the textbook
+// method: x = n + f with n = round(x), found by adding 1.5 * 2^23 (the sum's low mantissa bits then hold n)
+// and f = x - n in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients were fitted here to 2^f on
+// that interval by least squares with Lawson re-weighting toward the minimax fit (largest relative error
+// 7.5e-5, far below the 2^-9 of the bf16 the result is rounded to); 2^n is applied by adding n to the
+// exponent field.  Inputs below -125 (the masked keys' -inf included) are clamped to -125 so that the
+// exponent stays normal: they give 2^-125 instead of 0, which no sum in fp32 can tell apart.
+PA_DEVICE uint64_t exp2_poly2(uint64_t x2) {
+    constexpr float kShift = 12582912.f;          // 1.5 * 2^23
+    constexpr float c0 = 0.99992811f, c1 = 0.69326099f, c2 = 0.24261054f, c3 = 0.055171321f;
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t t = f2_add(xc, f2_pack(kShift, kShift));             // low mantissa bits: round(x)
+    const uint64_t r = f2_add(t, f2_pack(-kShift, -kShift));            // round(x) as a float
+    const uint64_t f = f2_fma(r, f2_pack(-1.f, -1.f), xc);              // x - round(x)
+    uint64_t p = f2_fma(f2_pack(c3, c3), f, f2_pack(c2, c2));
+    p = f2_fma(p, f, f2_pack(c1, c1));
+    p = f2_fma(p, f, f2_pack(c0, c0));
+    float p0, p1, t0, t1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(t, t0, t1);
+    // the shifter's own exponent and high mantissa bits vanish in the shift: t's bits << 23 == n << 23
+    const float y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    const float y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+    return f2_pack(y0, y1);
+}
+
+// max of three (sm_100 three-input max; NaN handling as fmaxf)
+PA_DEVICE float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a tile

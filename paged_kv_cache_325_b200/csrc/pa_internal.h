@@ -116,5 +116,6 @@ void set_last_error(pa_status status, const char *detail);
 
 // ------------------------------------------------------------- self-test --
 cudaError_t launch_selftest_wait(int32_t *dev_error, int64_t max_polls, cudaStream_t stream);
+cudaError_t launch_selftest_exp2(const float *x, float *y_poly, float *y_sfu, int32_t n, cudaStream_t stream);
 
 }  // namespace pa

@@ -51,7 +51,17 @@ constexpr int kN = 128;                // keys per K/V tile
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kFixWarp = 10;
-constexpr int kThreads = 352;          // 2 softmax warpgroups + TMA warp + MMA warp + V-fix warp
+constexpr int kThreads = 384;          // 2 softmax warpgroups + TMA warp + MMA warp + V-fix warp + warp 11, which
+                                       // has no role: it completes the third warpgroup for the register split
+// Register split (setmaxnreg): a 384-thread block is launched with kRegsAtLaunch registers per thread (the
+// most that ptxas gives it); the third warpgroup (TMA, MMA, V-fix, spare) drops to kRegsOther and the two
+// softmax warpgroups, which hold a 128-column S row and a 128-column O row per thread, rise to kRegsSoftmax.
+// The split must not ask for more than the block was launched with, or the increase waits forever: the
+// host checks the compiled register count before every first launch.
+constexpr uint32_t kRegsAtLaunch = 168;
+constexpr uint32_t kRegsOther = 136;
+constexpr uint32_t kRegsSoftmax = 184;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsAtLaunch, "register split");
 constexpr int kRowBytes = 128;         // one 64-element bf16 swizzle row
 constexpr int kSlab = kM * kRowBytes;  // 128 rows x 128 B = 16 KB
 constexpr int kUnitQueue = 4;          // unit ids handed from the TMA warp to the other roles
@@ -78,6 +88,13 @@ struct PrefillCfg {
                                                                 // (P_X, bf16, overwrites the first 64 columns of S_X)
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
+
+// Which pairs of a 32-key chunk take exp2 on the FMA pipe (exp2_poly2) rather than the special-function unit:
+// kPolyPairs of the 16, spread evenly.  ex2 on the special-function unit is the scarce resource of the
+// softmax (two 128-key rows per thread and key tile, one per Q tile); the polynomial costs about five
+// FMA-pipe instructions per element instead.
+constexpr int kPolyPairs = 0;
+__host__ __device__ constexpr bool poly_pair(int i) { return ((i + 1) * kPolyPairs) / 16 != (i * kPolyPairs) / 16; }
 
 __device__ __forceinline__ uint32_t col_s(int x) { return x ? 256u : 0u; }
 __device__ __forceinline__ uint32_t col_o(int x) { return x ? 384u : 128u; }
@@ -294,6 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *vlast_full = v_fixed + 1;           // [2]
     uint64_t *cp_full = vlast_full + 2;           // fused store: a copy round's rows are in the staging area
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
+    // set by the first wait of this CTA that gives up; every other wait then gives up at once
+    volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
     // unit queue: kUnitQueue entries of 16 words (a decoded Unit; valid = -1 ends the stream)
     volatile int32_t *unit_q = reinterpret_cast<volatile int32_t *>(tmem_slot + 16);
 
@@ -308,6 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t ring = sbase + C::kRingOff;
 
     if (threadIdx.x == 0) {
+        *abort_flag = 0;
         for (int i = 0; i < C::kSlots; ++i) {
             mbar_init(smem_u32(kv_full + i), 1);
             mbar_init(smem_u32(kv_empty + i), 1);
@@ -346,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // (valid = -1 ends the stream); the other roles pop them in order
     auto pop_unit = [&](uint32_t k, bool arrive, Unit &U) -> bool {
         const int slot = k % kUnitQueue;
-        if (!mbar_wait(smem_u32(uq_full + slot), (k / kUnitQueue) & 1, a.dev_error)) return false;
+        if (!mbar_wait(smem_u32(uq_full + slot), (k / kUnitQueue) & 1, a.dev_error, 0xffffffffu, abort_flag)) return false;
         int32_t *dst = reinterpret_cast<int32_t *>(&U);
 #pragma unroll
         for (int i = 0; i < 16; ++i) dst[i] = unit_q[slot * 16 + i];
@@ -355,80 +375,94 @@ __global__ void __launch_bounds__(kThreads, 1)
         return U.valid >= 0;
     };
 
-    if (warp == kTmaWarp) {
-        // ============================================================ TMA ==
-        // The whole warp runs this role: every lane waits on the barriers, lane 0 issues the copies, and
-        // block ids are read 32 at a time (one per lane) and passed around with shuffles.
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-        }
-        const int B = a.block_size, box = a.box_tokens;
-        const int total = plan_w[1];
-        const int4 *units = reinterpret_cast<const int4 *>(plan_w + plan.units);
-        const int4 *geo = reinterpret_cast<const int4 *>(plan_w + plan.geo);
-        auto fetch = [&]() -> int {
-            int u = 0;
-            if (lane == 0) u = (int)atomicAdd(reinterpret_cast<unsigned int *>(plan_w), 1u);
-            return __shfl_sync(0xffffffffu, u, 0);
-        };
-        auto decode = [&](int u) -> Unit {
-            Unit V;
-            if (u >= total) {
-                V.valid = -1;
-                return V;
-            }
-            const int4 rec = units[u];
-            return unit_from_record(a, rec, geo[rec.x], TQ);
-        };
-        uint32_t nq = 0, L = 0, nvlast = 0;
-        bool ok = true;
-        Unit next = decode(fetch());
-        for (uint32_t nu = 0;; ++nu) {
-            Unit U = next;
-            if (!ok) U.valid = -1;
-            const int slot = nu % kUnitQueue;
-            if (nu >= (uint32_t)kUnitQueue &&
-                !mbar_wait(smem_u32(uq_empty + slot), (nu / kUnitQueue - 1) & 1, a.dev_error))
-                U.valid = -1;
+    if (warp >= 8) {
+        // the third warpgroup (TMA, MMA and V-fix warps, and the spare warp, which has no role) gives
+        // registers back to the softmax warpgroups; all four warps run this one instruction
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+        if (warp == kTmaWarp) {
+            // ============================================================ TMA ==
+            // The whole warp runs this role: every lane waits on the barriers, lane 0 issues the copies, and
+            // block ids are read 32 at a time (one per lane) and passed around with shuffles.
             if (lane == 0) {
-                const int32_t *src = reinterpret_cast<const int32_t *>(&U);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) unit_q[slot * 16 + i] = src[i];
-                mbar_arrive(smem_u32(uq_full + slot));
+                tma_prefetch_desc(&tm_q);
+                tma_prefetch_desc(&tm_k);
+                tma_prefetch_desc(&tm_v);
             }
-            __syncwarp();
-            if (U.valid < 0) break;
-            // take the next unit now; its id and record loads overlap this unit's copies
-            const int next_u = fetch();
-            if (U.valid) {
-                if (nq > 0 && !mbar_wait(smem_u32(q_empty), (nq - 1) & 1, a.dev_error)) ok = false;
-                if (ok && lane == 0) {
-                    mbar_arrive_expect_tx(smem_u32(q_full), (uint32_t)(2 * C::kTileBytes));
-                    for (int x = 0; x < 2; ++x)
-#pragma unroll
-                        for (int h = 0; h < C::kHalves; ++h)
-                            tma_load_3d(q_s + x * C::kTileBytes + h * kSlab, &tm_q, h * 64, U.kvh * G,
-                                        U.q0 + U.tok0[x], smem_u32(q_full));
+            const int B = a.block_size, box = a.box_tokens;
+            const int total = plan_w[1];
+            const int4 *units = reinterpret_cast<const int4 *>(plan_w + plan.units);
+            const int4 *geo = reinterpret_cast<const int4 *>(plan_w + plan.geo);
+            auto fetch = [&]() -> int {
+                int u = 0;
+                if (lane == 0) u = (int)atomicAdd(reinterpret_cast<unsigned int *>(plan_w), 1u);
+                return __shfl_sync(0xffffffffu, u, 0);
+            };
+            auto decode = [&](int u) -> Unit {
+                Unit V;
+                if (u >= total) {
+                    V.valid = -1;
+                    return V;
                 }
-                if (ok) ++nq;
-                const int32_t *bt = a.block_table + (int64_t)U.s * a.bt_stride;
-                const int kend = max(U.kend[0], U.kend[1]);
-                int chunk = -32, ids = 0;            // block_table[chunk + lane] lives in `ids` of that lane
-                if (ok && U.nk > 0) ++nvlast;
-                for (int j = 0; j < U.nk && ok; ++j) {
-                    const int key0 = U.kbeg + j * kN;
-                    const int nbox = (min(kN, kend - key0) + box - 1) / box;
-                    const int last_blk = (key0 + (nbox - 1) * box) / B;
-                    if (last_blk >= chunk + 32) {
-                        chunk = key0 / B;
-                        ids = chunk + lane < a.bt_stride ? bt[chunk + lane] : -1;
-                    }
-                    for (int kv = 0; kv < 2 && ok; ++kv, ++L) {
+                const int4 rec = units[u];
+                return unit_from_record(a, rec, geo[rec.x], TQ);
+            };
+            uint32_t nq = 0, L = 0, nvlast = 0;
+            bool ok = true;
+            Unit next = decode(fetch());
+            for (uint32_t nu = 0;; ++nu) {
+                Unit U = next;
+                if (!ok) U.valid = -1;
+                const int slot = nu % kUnitQueue;
+                if (nu >= (uint32_t)kUnitQueue &&
+                    !mbar_wait(smem_u32(uq_empty + slot), (nu / kUnitQueue - 1) & 1, a.dev_error, 0xffffffffu, abort_flag))
+                    U.valid = -1;
+                if (lane == 0) {
+                    const int32_t *src = reinterpret_cast<const int32_t *>(&U);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) unit_q[slot * 16 + i] = src[i];
+                    mbar_arrive(smem_u32(uq_full + slot));
+                }
+                __syncwarp();
+                if (U.valid < 0) break;
+                // take the next unit now; its id and record loads overlap this unit's copies
+                const int next_u = fetch();
+                if (U.valid) {
+                    // Q first: the wait for the Q buffer (free once the previous unit's S products complete,
+                    // which the MMA thread issues only after the V fix of the unit before it) keeps this warp at
+                    // most one unit ahead of the V-fix warp, which the two alternating last-V barriers rely on.
+                    const int32_t *bt = a.block_table + (int64_t)U.s * a.bt_stride;
+                    const int kend = max(U.kend[0], U.kend[1]);
+                    int chunk = -32, ids = 0;            // block_table[chunk + lane] lives in `ids` of that lane
+                    if (ok && U.nk > 0) ++nvlast;
+                    const int nloads = 2 * U.nk, pre = 0;
+                    for (int li = 0; li <= nloads && ok; ++li) {
+                        if (li == pre) {
+                            if (nq > 0 && !mbar_wait(smem_u32(q_empty), (nq - 1) & 1, a.dev_error, 0xffffffffu, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            if (lane == 0) {
+                                mbar_arrive_expect_tx(smem_u32(q_full), (uint32_t)(2 * C::kTileBytes));
+                                for (int x = 0; x < 2; ++x)
+#pragma unroll
+                                    for (int h = 0; h < C::kHalves; ++h)
+                                        tma_load_3d(q_s + x * C::kTileBytes + h * kSlab, &tm_q, h * 64, U.kvh * G,
+                                                    U.q0 + U.tok0[x], smem_u32(q_full));
+                            }
+                            ++nq;
+                        }
+                        if (li == nloads) break;
+                        const int j = li >> 1, kv = li & 1;
+                        const int key0 = U.kbeg + j * kN;
+                        const int nbox = (min(kN, kend - key0) + box - 1) / box;
+                        const int last_blk = (key0 + (nbox - 1) * box) / B;
+                        if (last_blk >= chunk + 32) {
+                            chunk = key0 / B;
+                            ids = chunk + lane < a.bt_stride ? bt[chunk + lane] : -1;
+                        }
                         const int slot2 = L % C::kSlots;
                         if (L >= (uint32_t)C::kSlots &&
-                            !mbar_wait(smem_u32(kv_empty + slot2), (L / C::kSlots - 1) & 1, a.dev_error)) {
+                            !mbar_wait(smem_u32(kv_empty + slot2), (L / C::kSlots - 1) & 1, a.dev_error, 0xffffffffu, abort_flag)) {
                             ok = false;
                             break;
                         }
@@ -440,11 +474,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (vlast) mbar_arrive(smem_u32(kv_full + slot2));
                             mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * kRowBytes * C::kHalves));
                         }
+                        __syncwarp();                        // the expected bytes are posted before any copy
                         const uint32_t dst = ring + slot2 * C::kTileBytes;
-                        for (int b = 0; b < nbox; ++b) {
+                        // one box (block_size tokens, or 128 for larger blocks) per lane: with small blocks a
+                        // tile is many boxes, and one issuing thread would fall behind the tensor cores
+                        for (int b0 = 0; b0 < nbox; b0 += 32) {
+                            const int b = b0 + lane;
                             const int tok = key0 + b * box;
-                            const int blk = __shfl_sync(0xffffffffu, ids, tok / B - chunk);
-                            if (lane == 0) {
+                            const int blk = __shfl_sync(0xffffffffu, ids, b < nbox ? tok / B - chunk : 0);
+                            if (b < nbox) {
                                 int row;
                                 const CUtensorMap *map = kv ? &tm_v : &tm_k;
                                 if (kFused && tok >= U.c) {
@@ -463,283 +501,286 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     tma_load_3d(dst + h * kSlab + b * box * kRowBytes, map, h * 64, U.kvh, row, fb);
                             }
                         }
+                        ++L;
                     }
                 }
+                next = decode(next_u);
             }
-            next = decode(next_u);
-        }
-        // Leave no TMA copy in flight: wait (bounded) for the last load of every ring slot and for the
-        // last Q load.  On the normal path the MMA warp consumed them all and these return at once.
-        for (uint32_t i = (L > (uint32_t)C::kSlots ? L - C::kSlots : 0); i < L; ++i)
-            mbar_wait(smem_u32(kv_full + i % C::kSlots), (i / C::kSlots) & 1, a.dev_error);
-        if (nq > 0) mbar_wait(smem_u32(q_full), (nq - 1) & 1, a.dev_error);
-        for (uint32_t i = (nvlast > 2 ? nvlast - 2 : 0); i < nvlast; ++i)
-            mbar_wait(smem_u32(vlast_full + (i & 1)), (i >> 1) & 1, a.dev_error);
-    } else if (warp == kMmaWarp) {
-        // ============================================================ MMA ==
-        // One thread: the tensor cores keep almost no queue, so this thread does nothing but wait for
-        // its operands and issue.  Order per key tile j: PV_A(j) S_A(j+1) PV_B(j) S_B(j+1).
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kN, 0, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, D, 0, 1);
-            uint32_t nq = 0, L = 0, np[2] = {0, 0}, no[2] = {0, 0}, nfix = 0;
-            bool ok = true;
-            // Descriptors are built once; an MMA only adds a byte offset (>> 4) to the start-address
-            // field (14 bits of a 256 KB window, so the add never carries into the other fields).
-            const uint64_t q_desc = smem_desc_sw128(q_s, 16, 1024);
-            const uint64_t k_desc = smem_desc_sw128(ring, 16, 1024);
-            const uint64_t v_desc = smem_desc_sw128(ring, kSlab, 1024);
-            auto wait_slot = [&](uint32_t idx) -> bool {
-                return mbar_wait(smem_u32(kv_full + idx % C::kSlots), (idx / C::kSlots) & 1, a.dev_error);
-            };
-            auto issue_s = [&](int x, uint32_t kidx) {
-                const uint64_t qd = q_desc + ((uint32_t)(x * C::kTileBytes) >> 4);
-                const uint64_t kd = k_desc + (((kidx % C::kSlots) * (uint32_t)C::kTileBytes) >> 4);
-                const uint32_t d = tmem + col_s(x);
+            // Leave no TMA copy in flight: wait (bounded) for the last load of every ring slot and for the
+            // last Q load.  On the normal path the MMA warp consumed them all and these return at once; they
+            // ignore the abort flag, since the copies land in this CTA's shared memory whatever happened.
+            for (uint32_t i = (L > (uint32_t)C::kSlots ? L - C::kSlots : 0); i < L; ++i)
+                mbar_wait(smem_u32(kv_full + i % C::kSlots), (i / C::kSlots) & 1, a.dev_error);
+            if (nq > 0) mbar_wait(smem_u32(q_full), (nq - 1) & 1, a.dev_error);
+            for (uint32_t i = (nvlast > 2 ? nvlast - 2 : 0); i < nvlast; ++i)
+                mbar_wait(smem_u32(vlast_full + (i & 1)), (i >> 1) & 1, a.dev_error);
+        } else if (warp == kMmaWarp) {
+            // ============================================================ MMA ==
+            // One thread: the tensor cores keep almost no queue, so this thread does nothing but wait for
+            // its operands and issue.  Order per key tile j: PV_A(j) S_A(j+1) PV_B(j) S_B(j+1).
+            if (lane == 0) {
+                constexpr uint32_t idesc_qk = idesc_bf16_f32(kM, kN, 0, 0);
+                constexpr uint32_t idesc_pv = idesc_bf16_f32(kM, D, 0, 1);
+                uint32_t nq = 0, L = 0, np[2] = {0, 0}, no[2] = {0, 0}, nfix = 0;
+                bool ok = true;
+                // Descriptors are built once; an MMA only adds a byte offset (>> 4) to the start-address
+                // field (14 bits of a 256 KB window, so the add never carries into the other fields).
+                const uint64_t q_desc = smem_desc_sw128(q_s, 16, 1024);
+                const uint64_t k_desc = smem_desc_sw128(ring, 16, 1024);
+                const uint64_t v_desc = smem_desc_sw128(ring, kSlab, 1024);
+                auto wait_slot = [&](uint32_t idx) -> bool {
+                    return mbar_wait(smem_u32(kv_full + idx % C::kSlots), (idx / C::kSlots) & 1, a.dev_error, 0xffffffffu, abort_flag);
+                };
+                auto issue_s = [&](int x, uint32_t kidx) {
+                    const uint64_t qd = q_desc + ((uint32_t)(x * C::kTileBytes) >> 4);
+                    const uint64_t kd = k_desc + (((kidx % C::kSlots) * (uint32_t)C::kTileBytes) >> 4);
+                    const uint32_t d = tmem + col_s(x);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * kSlab + (kk & 3) * 32) >> 4;
-                    tc_mma_ss(d, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
-                }
-                tc_commit(smem_u32(s_full + x));
-            };
-            auto issue_pv = [&](int x, uint32_t vidx, bool accumulate) {
-                const uint64_t vd = v_desc + (((vidx % C::kSlots) * (uint32_t)C::kTileBytes) >> 4);
-                const uint32_t d = tmem + col_o(x), pa = tmem + col_s(x);
-#pragma unroll
-                for (int kk = 0; kk < kN / 16; ++kk) {
-                    // A = P_X in TMEM: 16 keys = 8 columns of packed bf16 pairs; B = V rows kk*16 ..
-                    tc_mma_ts(d, pa + kk * 8, vd + ((kk * 16 * kRowBytes) >> 4), idesc_pv,
-                              (accumulate || kk > 0) ? 1u : 0u);
-                }
-            };
-            for (uint32_t k = 0; ok; ++k) {
-                const int slot = k % kUnitQueue;
-                if (!mbar_wait(smem_u32(uq_full + slot), (k / kUnitQueue) & 1, a.dev_error)) break;
-                Unit U;
-                {
-                    int32_t *dst = reinterpret_cast<int32_t *>(&U);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) dst[i] = unit_q[slot * 16 + i];
-                }
-                mbar_arrive(smem_u32(uq_empty + slot));
-                if (U.valid < 0) break;
-                if (!U.valid) continue;
-                if (!mbar_wait(smem_u32(q_full), nq & 1, a.dev_error)) break;
-                ++nq;
-                const bool hasB = U.nt[1] > 0;
-                // K_0: S_A(0), S_B(0)
-                if (!wait_slot(L)) break;
-                tc_fence_after();
-                issue_s(0, L);
-                if (hasB) issue_s(1, L);
-                tc_commit(smem_u32(kv_empty + L % C::kSlots));
-                if (U.nk == 1) tc_commit(smem_u32(q_empty));
-                for (int j = 0; j < U.nk && ok; ++j) {
-                    const uint32_t vidx = L + 2 * j + 1, knext = L + 2 * j + 2;
-                    if (j == U.nk - 1) {
-                        // the V-fix warp has zeroed the rows past the key range of the unit's last V tile
-                        if (!mbar_wait(smem_u32(v_fixed), nfix & 1, a.dev_error)) { ok = false; break; }
-                        ++nfix;
-                    } else if (!wait_slot(vidx)) {
-                        ok = false;
-                        break;
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk >> 2) * kSlab + (kk & 3) * 32) >> 4;
+                        tc_mma_ss(d, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
                     }
-                    bool knext_ready = false;
-                    for (int x = 0; x < 2; ++x) {
-                        if (j >= U.nt[x]) continue;
-                        if (!mbar_wait(smem_u32(p_full + x), np[x] & 1, a.dev_error)) { ok = false; break; }
-                        ++np[x];
-                        if (j == 0 && no[x] > 0 &&
-                            !mbar_wait(smem_u32(o_empty + x), (no[x] - 1) & 1, a.dev_error)) {
+                    tc_commit(smem_u32(s_full + x));
+                };
+                auto issue_pv = [&](int x, uint32_t vidx, bool accumulate) {
+                    const uint64_t vd = v_desc + (((vidx % C::kSlots) * (uint32_t)C::kTileBytes) >> 4);
+                    const uint32_t d = tmem + col_o(x), pa = tmem + col_s(x);
+#pragma unroll
+                    for (int kk = 0; kk < kN / 16; ++kk) {
+                        // A = P_X in TMEM: 16 keys = 8 columns of packed bf16 pairs; B = V rows kk*16 ..
+                        tc_mma_ts(d, pa + kk * 8, vd + ((kk * 16 * kRowBytes) >> 4), idesc_pv,
+                                  (accumulate || kk > 0) ? 1u : 0u);
+                    }
+                };
+                for (uint32_t k = 0; ok; ++k) {
+                    const int slot = k % kUnitQueue;
+                    if (!mbar_wait(smem_u32(uq_full + slot), (k / kUnitQueue) & 1, a.dev_error, 0xffffffffu, abort_flag)) break;
+                    Unit U;
+                    {
+                        int32_t *dst = reinterpret_cast<int32_t *>(&U);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) dst[i] = unit_q[slot * 16 + i];
+                    }
+                    mbar_arrive(smem_u32(uq_empty + slot));
+                    if (U.valid < 0) break;
+                    if (!U.valid) continue;
+                    if (!mbar_wait(smem_u32(q_full), nq & 1, a.dev_error, 0xffffffffu, abort_flag)) break;
+                    ++nq;
+                    const bool hasB = U.nt[1] > 0;
+                    // K_0: S_A(0), S_B(0)
+                    if (!wait_slot(L)) break;
+                    tc_fence_after();
+                    issue_s(0, L);
+                    if (hasB) issue_s(1, L);
+                    tc_commit(smem_u32(kv_empty + L % C::kSlots));
+                    if (U.nk == 1) tc_commit(smem_u32(q_empty));
+                    for (int j = 0; j < U.nk && ok; ++j) {
+                        const uint32_t vidx = L + 2 * j + 1, knext = L + 2 * j + 2;
+                        if (j == U.nk - 1) {
+                            // the V-fix warp has zeroed the rows past the key range of the unit's last V tile
+                            if (!mbar_wait(smem_u32(v_fixed), nfix & 1, a.dev_error, 0xffffffffu, abort_flag)) { ok = false; break; }
+                            ++nfix;
+                        } else if (!wait_slot(vidx)) {
                             ok = false;
                             break;
                         }
-                        tc_fence_after();
-                        issue_pv(x, vidx, j > 0);
-                        if (j == U.nt[x] - 1) {
-                            tc_commit(smem_u32(o_full + x));
-                            ++no[x];
-                        }
-                        if (j + 1 < U.nt[x]) {
-                            if (!knext_ready) {
-                                if (!wait_slot(knext)) { ok = false; break; }
-                                tc_fence_after();
-                                knext_ready = true;
+                        bool knext_ready = false;
+                        for (int x = 0; x < 2; ++x) {
+                            if (j >= U.nt[x]) continue;
+                            if (!mbar_wait(smem_u32(p_full + x), np[x] & 1, a.dev_error, 0xffffffffu, abort_flag)) { ok = false; break; }
+                            ++np[x];
+                            if (j == 0 && no[x] > 0 &&
+                                !mbar_wait(smem_u32(o_empty + x), (no[x] - 1) & 1, a.dev_error, 0xffffffffu, abort_flag)) {
+                                ok = false;
+                                break;
                             }
-                            issue_s(x, knext);
+                            tc_fence_after();
+                            issue_pv(x, vidx, j > 0);
+                            if (j == U.nt[x] - 1) {
+                                tc_commit(smem_u32(o_full + x));
+                                ++no[x];
+                            }
+                            if (j + 1 < U.nt[x]) {
+                                if (!knext_ready) {
+                                    if (!wait_slot(knext)) { ok = false; break; }
+                                    tc_fence_after();
+                                    knext_ready = true;
+                                }
+                                issue_s(x, knext);
+                            }
                         }
+                        if (!ok) break;
+                        tc_commit(smem_u32(kv_empty + vidx % C::kSlots));
+                        if (knext_ready) tc_commit(smem_u32(kv_empty + knext % C::kSlots));
+                        if (j == U.nk - 2) tc_commit(smem_u32(q_empty));   // every S product of the unit is issued
                     }
-                    if (!ok) break;
-                    tc_commit(smem_u32(kv_empty + vidx % C::kSlots));
-                    if (knext_ready) tc_commit(smem_u32(kv_empty + knext % C::kSlots));
-                    if (j == U.nk - 2) tc_commit(smem_u32(q_empty));   // every S product of the unit is issued
+                    L += 2 * U.nk;
                 }
-                L += 2 * U.nk;
+                // every MMA issued by this thread has completed before TMEM is freed
+                tc_commit(smem_u32(done));
+                mbar_wait(smem_u32(done), 0, a.dev_error);
             }
-            // every MMA issued by this thread has completed before TMEM is freed
-            tc_commit(smem_u32(done));
-            mbar_wait(smem_u32(done), 0, a.dev_error);
-        }
-    } else if (warp == kFixWarp) {
-        // ========================================================== V fix ==
-        // Zero the rows of each unit's last V tile past its key range (stale or poisoned cache slots),
-        // so that masked keys, whose probabilities are exactly 0, never meet a NaN.
-        // Fused store: between those fixes this warp copies each unit's own new tokens' K/V rows of its KV
-        // head to their cache slots with the bulk-copy engine, in rounds of up to kStageTokens tokens:
-        // bulk loads of the rows into the staging area (completing on cp_full), then one bulk store per
-        // row to its slot.  The warp never waits on a copy while a fix is due -- it polls for the next
-        // unit's last V tile between steps -- so the MMA waits for fixes only.  Units whose rows are not
-        // yet copied wait in a small FIFO; the rest is copied when the CTA has no unit left.  No kernel of
-        // this launch reads those slots.
-        uint32_t L = 0, nfx = 0;
-        constexpr int kFifo = 4;
-        int fq_s[kFifo], fq_kvh[kFifo], fq_q0[kFifo], fq_c[kFifo], fq_i[kFifo], fq_end[kFifo];
-        int fq_head = 0, fq_n = 0;            // oldest entry, entries in use
-        int cp_state = 0;                     // 0: staging free, 1: loads in flight, 2: stores issued
-        uint32_t cp_rounds = 0;               // completed phases of cp_full
-        int rd_s = 0, rd_kvh = 0, rd_q0 = 0, rd_c = 0, rd_i = 0, rd_n = 0;   // the round in flight
-        const uint32_t stage = sbase + C::kStageOff;
-        const uint32_t cpb = smem_u32(cp_full);
-        // take up to kStageTokens tokens of the oldest pending unit and start their loads
-        auto start_round = [&]() {
-            int end = 0;
-#pragma unroll
-            for (int e = 0; e < kFifo; ++e)
-                if (e == fq_head) {
-                    rd_s = fq_s[e];
-                    rd_kvh = fq_kvh[e];
-                    rd_q0 = fq_q0[e];
-                    rd_c = fq_c[e];
-                    rd_i = fq_i[e];
-                    end = fq_end[e];
-                }
-            rd_n = min(C::kStageTokens, end - rd_i);
-#pragma unroll
-            for (int e = 0; e < kFifo; ++e)
-                if (e == fq_head) fq_i[e] = rd_i + rd_n;
-            if (rd_i + rd_n >= end) {
-                fq_head = (fq_head + 1) % kFifo;
-                --fq_n;
-            }
-            if (lane == 0) mbar_arrive_expect_tx(cpb, (uint32_t)(rd_n * 4 * D));
-            __syncwarp();
-            for (int t = lane; t < rd_n; t += 32) {
-                const int64_t row = (int64_t)rd_q0 + rd_i + t;
-                bulk_load(stage + t * 4 * D,
-                          static_cast<const __nv_bfloat16 *>(a.k_new) + row * a.kn_stride + (int64_t)rd_kvh * D, 2 * D,
-                          cpb);
-                bulk_load(stage + t * 4 * D + 2 * D,
-                          static_cast<const __nv_bfloat16 *>(a.v_new) + row * a.vn_stride + (int64_t)rd_kvh * D, 2 * D,
-                          cpb);
-            }
-            cp_state = 1;
-        };
-        // the round's rows have landed: one bulk store per row to its slot
-        auto store_round = [&]() {
-            mbar_wait(cpb, cp_rounds & 1, a.dev_error);   // returns at once: every lane acquires the rows
-            ++cp_rounds;
-            for (int t = lane; t < rd_n; t += 32) {
-                const int64_t row = (int64_t)rd_q0 + rd_i + t;
-                const int32_t sl = __ldg(a.new_slots + row);
-                if (sl < 0 || (int64_t)sl >= a.num_slots) {
-                    report(a.dev_error, PA_DEVERR_SLOT);   // not stored
-                    continue;
-                }
-                if (a.dev_error) {   // the slot must be the row this prefill read as key c + i
-                    const int pos = rd_c + rd_i + t;
-                    const int32_t blk = __ldg(a.block_table + (int64_t)rd_s * a.bt_stride + pos / a.block_size);
-                    if ((int64_t)sl != (int64_t)blk * a.block_size + pos % a.block_size) report(a.dev_error, PA_DEVERR_SLOT);
-                }
-                const int64_t off = ((int64_t)sl * a.num_kv_heads + rd_kvh) * D;
-                bulk_store(static_cast<__nv_bfloat16 *>(a.k_cache) + off, stage + t * 4 * D, 2 * D);
-                bulk_store(static_cast<__nv_bfloat16 *>(a.v_cache) + off, stage + t * 4 * D + 2 * D, 2 * D);
-            }
-            bulk_commit();
-            cp_state = 2;
-        };
-        // One loop, one site for each copy step.  With no unit left it drains the FIFO.
-        bool more = true;
-        for (uint32_t k = 0;; ++k) {
-            Unit U;
-            U.valid = 0;
-            if (more && !pop_unit(k, lane == 0, U)) more = false;
-            if (more && !U.valid) continue;
-            const uint32_t vbar = smem_u32(vlast_full + (nfx & 1)), vpar = (nfx >> 1) & 1;
-            if (kFused) {
-                // pump the copy engine until the unit's last V tile lands (a fix first, always) or, with
-                // no unit left, until nothing is pending; leave room in the FIFO for this unit.  Bounded:
-                // polls sleep 128 ns and a round's loads are waited for at most kWaitTimeoutNs.
-                uint64_t t_loads = 0;
-                for (;;) {
-                    if (more && fq_n < kFifo && __any_sync(0xffffffffu, mbar_test_wait(vbar, vpar))) break;
-                    if (cp_state == 1) {
-                        const bool landed = __any_sync(0xffffffffu, mbar_test_wait(cpb, cp_rounds & 1));
-                        if (landed || !more || (t_loads && global_timer_ns() - t_loads > kWaitTimeoutNs)) {
-                            store_round();
-                            t_loads = 0;
-                        } else {
-                            if (!t_loads) t_loads = global_timer_ns();
-                            __nanosleep(128);
-                        }
-                        continue;
-                    }
-                    if (cp_state == 2) {          // the staging area is free once the stores have read it
-                        bulk_wait_read();
-                        __syncwarp();
-                        cp_state = 0;
-                        continue;
-                    }
-                    if (fq_n > 0) {
-                        start_round();
-                        continue;
-                    }
-                    break;                        // nothing pending
-                }
-            }
-            if (!more) break;
-            const uint32_t vidx = L + 2 * (U.nk - 1) + 1;
-            L += 2 * U.nk;
-            if (!mbar_wait(vbar, vpar, a.dev_error)) break;
-            ++nfx;
-            const int valid = max(U.kend[0], U.kend[1]) - (U.kbeg + (U.nk - 1) * kN);
-            if (valid < kN) {
-                const uint32_t vs = ring + (vidx % C::kSlots) * C::kTileBytes;
-                for (int e = lane; e < (kN - valid) * C::kHalves * 8; e += 32) {
-                    const int r = valid + e / (C::kHalves * 8);
-                    const int h = (e / 8) % C::kHalves, ch = e % 8;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(vs + h * kSlab + r * kRowBytes + ch * 16),
-                                 "r"(0u)
-                                 : "memory");
-                }
-                fence_proxy_async_smem();
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(v_fixed));
-            if (kFused && U.chunk == 0) {
-                // this unit's own tokens: tile A's, then tile B's (present only when tile A is full); the
-                // loop above left room in the FIFO
-                const int e_new = (fq_head + fq_n) % kFifo;
-                const int i0 = U.tok0[0], i1 = min(U.n_new, U.tok0[0] + 2 * TQ);
+        } else if (warp == kFixWarp) {
+            // ========================================================== V fix ==
+            // Zero the rows of each unit's last V tile past its key range (stale or poisoned cache slots),
+            // so that masked keys, whose probabilities are exactly 0, never meet a NaN.
+            // Fused store: between those fixes this warp copies each unit's own new tokens' K/V rows of its KV
+            // head to their cache slots with the bulk-copy engine, in rounds of up to kStageTokens tokens:
+            // bulk loads of the rows into the staging area (completing on cp_full), then one bulk store per
+            // row to its slot.  The warp never waits on a copy while a fix is due -- it polls for the next
+            // unit's last V tile between steps -- so the MMA waits for fixes only.  Units whose rows are not
+            // yet copied wait in a small FIFO; the rest is copied when the CTA has no unit left.  No kernel of
+            // this launch reads those slots.
+            uint32_t L = 0, nfx = 0;
+            constexpr int kFifo = 4;
+            int fq_s[kFifo], fq_kvh[kFifo], fq_q0[kFifo], fq_c[kFifo], fq_i[kFifo], fq_end[kFifo];
+            int fq_head = 0, fq_n = 0;            // oldest entry, entries in use
+            int cp_state = 0;                     // 0: staging free, 1: loads in flight, 2: stores issued
+            uint32_t cp_rounds = 0;               // completed phases of cp_full
+            int rd_s = 0, rd_kvh = 0, rd_q0 = 0, rd_c = 0, rd_i = 0, rd_n = 0;   // the round in flight
+            const uint32_t stage = sbase + C::kStageOff;
+            const uint32_t cpb = smem_u32(cp_full);
+            // take up to kStageTokens tokens of the oldest pending unit and start their loads
+            auto start_round = [&]() {
+                int end = 0;
 #pragma unroll
                 for (int e = 0; e < kFifo; ++e)
-                    if (e == e_new) {
-                        fq_s[e] = U.s;
-                        fq_kvh[e] = U.kvh;
-                        fq_q0[e] = U.q0;
-                        fq_c[e] = U.c;
-                        fq_i[e] = i0;
-                        fq_end[e] = i1;
+                    if (e == fq_head) {
+                        rd_s = fq_s[e];
+                        rd_kvh = fq_kvh[e];
+                        rd_q0 = fq_q0[e];
+                        rd_c = fq_c[e];
+                        rd_i = fq_i[e];
+                        end = fq_end[e];
                     }
-                if (i1 > i0) ++fq_n;
+                rd_n = min(C::kStageTokens, end - rd_i);
+#pragma unroll
+                for (int e = 0; e < kFifo; ++e)
+                    if (e == fq_head) fq_i[e] = rd_i + rd_n;
+                if (rd_i + rd_n >= end) {
+                    fq_head = (fq_head + 1) % kFifo;
+                    --fq_n;
+                }
+                if (lane == 0) mbar_arrive_expect_tx(cpb, (uint32_t)(rd_n * 4 * D));
+                __syncwarp();
+                for (int t = lane; t < rd_n; t += 32) {
+                    const int64_t row = (int64_t)rd_q0 + rd_i + t;
+                    bulk_load(stage + t * 4 * D,
+                              static_cast<const __nv_bfloat16 *>(a.k_new) + row * a.kn_stride + (int64_t)rd_kvh * D, 2 * D,
+                              cpb);
+                    bulk_load(stage + t * 4 * D + 2 * D,
+                              static_cast<const __nv_bfloat16 *>(a.v_new) + row * a.vn_stride + (int64_t)rd_kvh * D, 2 * D,
+                              cpb);
+                }
+                cp_state = 1;
+            };
+            // the round's rows have landed: one bulk store per row to its slot
+            auto store_round = [&]() {
+                mbar_wait(cpb, cp_rounds & 1, a.dev_error);   // returns at once: every lane acquires the rows
+                ++cp_rounds;
+                for (int t = lane; t < rd_n; t += 32) {
+                    const int64_t row = (int64_t)rd_q0 + rd_i + t;
+                    const int32_t sl = __ldg(a.new_slots + row);
+                    if (sl < 0 || (int64_t)sl >= a.num_slots) {
+                        report(a.dev_error, PA_DEVERR_SLOT);   // not stored
+                        continue;
+                    }
+                    if (a.dev_error) {   // the slot must be the row this prefill read as key c + i
+                        const int pos = rd_c + rd_i + t;
+                        const int32_t blk = __ldg(a.block_table + (int64_t)rd_s * a.bt_stride + pos / a.block_size);
+                        if ((int64_t)sl != (int64_t)blk * a.block_size + pos % a.block_size) report(a.dev_error, PA_DEVERR_SLOT);
+                    }
+                    const int64_t off = ((int64_t)sl * a.num_kv_heads + rd_kvh) * D;
+                    bulk_store(static_cast<__nv_bfloat16 *>(a.k_cache) + off, stage + t * 4 * D, 2 * D);
+                    bulk_store(static_cast<__nv_bfloat16 *>(a.v_cache) + off, stage + t * 4 * D + 2 * D, 2 * D);
+                }
+                bulk_commit();
+                cp_state = 2;
+            };
+            // One loop, one site for each copy step.  With no unit left it drains the FIFO.
+            bool more = true;
+            for (uint32_t k = 0;; ++k) {
+                Unit U;
+                U.valid = 0;
+                if (more && !pop_unit(k, lane == 0, U)) more = false;
+                if (more && !U.valid) continue;
+                const uint32_t vbar = smem_u32(vlast_full + (nfx & 1)), vpar = (nfx >> 1) & 1;
+                if (kFused) {
+                    // pump the copy engine until the unit's last V tile lands (a fix first, always) or, with
+                    // no unit left, until nothing is pending; leave room in the FIFO for this unit.  Bounded:
+                    // polls sleep 128 ns and a round's loads are waited for at most kWaitTimeoutNs.
+                    uint64_t t_loads = 0;
+                    for (;;) {
+                        if (more && fq_n < kFifo && __any_sync(0xffffffffu, mbar_test_wait(vbar, vpar))) break;
+                        if (cp_state == 1) {
+                            const bool landed = __any_sync(0xffffffffu, mbar_test_wait(cpb, cp_rounds & 1));
+                            if (landed || !more || (t_loads && global_timer_ns() - t_loads > kWaitTimeoutNs)) {
+                                store_round();
+                                t_loads = 0;
+                            } else {
+                                if (!t_loads) t_loads = global_timer_ns();
+                                __nanosleep(128);
+                            }
+                            continue;
+                        }
+                        if (cp_state == 2) {          // the staging area is free once the stores have read it
+                            bulk_wait_read();
+                            __syncwarp();
+                            cp_state = 0;
+                            continue;
+                        }
+                        if (fq_n > 0) {
+                            start_round();
+                            continue;
+                        }
+                        break;                        // nothing pending
+                    }
+                }
+                if (!more) break;
+                const uint32_t vidx = L + 2 * (U.nk - 1) + 1;
+                L += 2 * U.nk;
+                if (!mbar_wait(vbar, vpar, a.dev_error, 0xffffffffu, abort_flag)) break;
+                ++nfx;
+                const int valid = max(U.kend[0], U.kend[1]) - (U.kbeg + (U.nk - 1) * kN);
+                if (valid < kN) {
+                    const uint32_t vs = ring + (vidx % C::kSlots) * C::kTileBytes;
+                    for (int e = lane; e < (kN - valid) * C::kHalves * 8; e += 32) {
+                        const int r = valid + e / (C::kHalves * 8);
+                        const int h = (e / 8) % C::kHalves, ch = e % 8;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(vs + h * kSlab + r * kRowBytes + ch * 16),
+                                     "r"(0u)
+                                     : "memory");
+                    }
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(v_fixed));
+                if (kFused && U.chunk == 0) {
+                    // this unit's own tokens: tile A's, then tile B's (present only when tile A is full); the
+                    // loop above left room in the FIFO
+                    const int e_new = (fq_head + fq_n) % kFifo;
+                    const int i0 = U.tok0[0], i1 = min(U.n_new, U.tok0[0] + 2 * TQ);
+#pragma unroll
+                    for (int e = 0; e < kFifo; ++e)
+                        if (e == e_new) {
+                            fq_s[e] = U.s;
+                            fq_kvh[e] = U.kvh;
+                            fq_q0[e] = U.q0;
+                            fq_c[e] = U.c;
+                            fq_i[e] = i0;
+                            fq_end[e] = i1;
+                        }
+                    if (i1 > i0) ++fq_n;
+                }
+            }
+            if (kFused) {
+                // leave nothing in flight: the last round's loads (bounded), then every bulk store
+                if (cp_state == 1) mbar_wait(cpb, cp_rounds & 1, a.dev_error);
+                bulk_wait_all();
             }
         }
-        if (kFused) {
-            // leave nothing in flight: the last round's loads (bounded), then every bulk store
-            if (cp_state == 1) mbar_wait(cpb, cp_rounds & 1, a.dev_error);
-            bulk_wait_all();
-        }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         // ======================================================== softmax ==
         const int x = warp >> 2;                       // 0: tile A, 1: tile B
         const int r = threadIdx.x & 127;               // TMEM lane == Q-tile row
@@ -756,7 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float m_ref = -INFINITY, l = 0.f;
             bool ok = true;
             for (int j = 0; j < U.nt[x]; ++j) {
-                if (!mbar_wait(smem_u32(s_full + x), ns & 1, a.dev_error)) { ok = false; break; }
+                if (!mbar_wait(smem_u32(s_full + x), ns & 1, a.dev_error, 0xffffffffu, abort_flag)) { ok = false; break; }
                 ++ns;
                 tc_fence_after();
                 uint32_t sr[4][32];
@@ -764,19 +805,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int q = 0; q < 4; ++q) tmem_ld32(lane_base + col_s(x) + q * 32, sr[q]);
                 tc_wait_ld();
                 const int thr = lim - (U.kbeg + j * kN);   // keys e <= thr are visible
-                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                // row maximum: three-input max over pairs, eight independent chains
+                float mx[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) mx[c] = -INFINITY;
                 if (thr >= kN - 1) {
 #pragma unroll
-                    for (int e = 0; e < kN; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(sr[e >> 5][e & 31]));
+                    for (int e = 0; e < kN; e += 16)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            mx[c] = max3f(mx[c], __uint_as_float(sr[(e + 2 * c) >> 5][(e + 2 * c) & 31]),
+                                          __uint_as_float(sr[(e + 2 * c + 1) >> 5][(e + 2 * c + 1) & 31]));
                 } else {
 #pragma unroll
                     for (int e = 0; e < kN; ++e) {
                         const float v = e <= thr ? __uint_as_float(sr[e >> 5][e & 31]) : -INFINITY;
                         sr[e >> 5][e & 31] = __float_as_uint(v);
-                        mx[e & 3] = fmaxf(mx[e & 3], v);
+                        mx[e & 7] = fmaxf(mx[e & 7], v);
                     }
                 }
-                const float m_new = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl;
+                const float m_new =
+                    fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], max3f(mx[5], mx[6], mx[7]))) * sl;
                 float corr = 1.f;
                 bool rescale = false;
                 if (m_new > m_ref + 8.f) {                  // also true while m_ref is -inf
@@ -784,23 +833,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_ref = m_new;
                     rescale = true;
                 }
-                const float neg = -m_ref;
                 // P = exp2(s * scale_log2 - m_ref) as packed bf16 pairs, written over the S_X columns already
-                // read (32 keys = 16 columns per store)
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                // read (32 keys = 16 columns per store); the scaling runs on pairs (f32x2 FMA).  The row sum
+                // adds the bf16 values the PV product multiplies, not the fp32 ones, so that the weights of the
+                // numerator and the denominator are the same numbers: with the lazy maximum the largest P is not
+                // a power of two, and its rounding would otherwise show in the output of a row that one key
+                // dominates.
+                const uint64_t sl2 = f2_pack(sl, sl), neg2 = f2_pack(-m_ref, -m_ref);
+                uint64_t ls2[2] = {0ull, 0ull};
 #pragma unroll
                 for (int kc = 0; kc < kN / 32; ++kc) {
                     uint32_t w[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const int e = kc * 32 + 2 * i;
-                        const float p0 = fast_exp2(fmaf(__uint_as_float(sr[e >> 5][e & 31]), sl, neg));
-                        const float p1 = fast_exp2(fmaf(__uint_as_float(sr[e >> 5][(e + 1) & 31]), sl, neg));
+                        const uint64_t x2 =
+                            f2_fma(f2_pack(__uint_as_float(sr[kc][2 * i]), __uint_as_float(sr[kc][2 * i + 1])), sl2, neg2);
+                        float p0, p1;
+                        if (poly_pair(i)) {
+                            f2_unpack(exp2_poly2(x2), p0, p1);
+                        } else {
+                            f2_unpack(x2, p0, p1);
+                            p0 = fast_exp2(p0);
+                            p1 = fast_exp2(p1);
+                        }
                         w[i] = pack_bf16(p0, p1);
-                        ls[i & 3] += p0 + p1;
+                        ls2[i & 1] = f2_add(ls2[i & 1], f2_pack(__uint_as_float(w[i] << 16),
+                                                                __uint_as_float(w[i] & 0xffff0000u)));
                     }
                     tmem_st16(lane_base + col_s(x) + kc * 16, w);
                 }
+                float ls[4];
+                f2_unpack(ls2[0], ls[0], ls[1]);
+                f2_unpack(ls2[1], ls[2], ls[3]);
                 l = l * corr + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
                 // The decision is per row, but tcgen05.ld / st are warp-wide (.sync.aligned): the whole warp
                 // takes the branch when any of its rows rescales, and the other rows multiply by corr = 1.
@@ -824,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             // ---- epilogue: O / l -> bf16 rows ----
-            if (!mbar_wait(smem_u32(o_full + x), no & 1, a.dev_error)) break;
+            if (!mbar_wait(smem_u32(o_full + x), no & 1, a.dev_error, 0xffffffffu, abort_flag)) break;
             ++no;
             tc_fence_after();
             const float inv = 1.f / l;
@@ -836,6 +900,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q = 0; q < D / 32; ++q) tmem_ld32(lane_base + col_o(x) + q * 32, o[q]);
             tc_wait_ld();
+            // O_X is in registers: hand its TMEM columns back to the MMA thread now, so that the next unit's
+            // first PV product does not wait for the global stores below
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(o_empty + x));
             if (store && a.part_o) {
                 // partial result of this key chunk: fp32 O / l and its log-sum-exp (log2 units), to be merged
                 // with the other partials of the same (query, head)
@@ -862,9 +931,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         dst[(q * 32 + e) / 8] = v;
                     }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(o_empty + x));
         }
     }
 
@@ -896,6 +962,11 @@ cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &tm_q, cons
     if (e != cudaSuccess) return e;
     const uint64_t bit = uint64_t(1) << (dev & 63);
     if (!(configured[fused].load(std::memory_order_acquire) & bit)) {
+        // the register split inside the kernel assumes the launch-time count it was written for
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, kernel);
+        if (e != cudaSuccess) return e;
+        if ((uint32_t)fa.numRegs * kThreads < 2 * 128 * kRegsSoftmax + 128 * kRegsOther) return cudaErrorNotSupported;
         e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
         if (e != cudaSuccess) return e;
         configured[fused].fetch_or(bit, std::memory_order_acq_rel);

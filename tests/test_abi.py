@@ -186,6 +186,9 @@ def test_prefill_validation(lib):
 
 
 def test_selftest_validation(lib):
+    assert lib.pa_selftest_exp2(None, None, None, 4, None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_selftest_exp2(None, None, None, -1, None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_selftest_exp2(None, None, None, 0, None) == pa.PA_OK
     assert lib.pa_selftest_bounded_wait(None, 100, None) == pa.PA_ERR_INVALID_ARG
     assert lib.pa_selftest_bounded_wait(A, 0, None) == pa.PA_ERR_INVALID_ARG
 

@@ -95,6 +95,7 @@ constexpr int kPlanHdrBytes = 256;
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBuckets = 1024;          // item lengths (tiles) for the longest-first order; longer share the last
 constexpr int kPlanCache = 2048;            // sequences whose length the planning kernel keeps in shared memory
+constexpr int kPlanSplitList = 1024;        // split (sequence, KV head) pairs whose items a warp each writes
 
 // Context length of sequence s: context_lens[s]; in the varlen mode (the decode rows of a mixed batch) the
 // key count of a sequence with exactly one new token, and -1 for any other sequence (not this call's work).
@@ -154,9 +155,8 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
     if ((tid & 31) == 0) atomicAdd(&s_total, part);
     __syncthreads();
-    // split rule: pairs up to the average per-CTA load stay whole; longer ones are cut into pieces of a
-    // sixteenth of it (never finer than the host's chunk, which sized the partial slots), so that the last
-    // pieces handed out -- and with them the spread of the CTAs' finishing times -- stay short
+    // split rule: pairs up to the average per-CTA load stay whole; longer ones are cut into pieces of an
+    // eighth of it (never finer than the host's chunk, which sized the partial slots)
     int whole, chunk;
     const int host_chunk = a.plan.chunk / kTile;
     if (a.plan.fixed) {
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         const unsigned long long avg = (s_total + num_ctas - 1) / (unsigned long long)num_ctas;
         whole = (int)min(avg, 1ull << 30);
         if (whole < 4) whole = 4;
-        chunk = (int)min((avg + 15) / 16, 1ull << 30);
+        chunk = (int)min((avg + 7) / 8, 1ull << 30);
         if (chunk < host_chunk) chunk = host_chunk;
     }
     // longest-first order: count items per length bucket, then exclusive offsets from the longest bucket
@@ -240,9 +240,14 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         }
     }
     int4 *items = reinterpret_cast<int4 *>(reinterpret_cast<char *>(a.plan_ws) + kPlanHdrBytes);
-    const int64_t npairs = (int64_t)a.batch * a.num_kv_heads;
-    for (int64_t pr = tid; pr < npairs; pr += kPlanThreads) {
-        const int s = (int)(pr / a.num_kv_heads), kvh = (int)(pr % a.num_kv_heads);
+    const int npairs = a.batch * a.num_kv_heads;     // < 2^31: the host bounds batch and KV heads
+    // whole pairs: one thread each; split pairs go to a list (or, past its capacity, are written here)
+    __shared__ int s_split[kPlanSplitList];
+    __shared__ int s_nsplit;
+    if (tid == 0) s_nsplit = 0;
+    __syncthreads();
+    for (int pr = tid; pr < npairs; pr += kPlanThreads) {
+        const int s = pr / a.num_kv_heads, kvh = pr - s * a.num_kv_heads;
         const int tiles = s < kPlanCache ? s_tiles[s] : dec_tiles(a, s, false);
         const int n = dec_nsplit(tiles, whole, chunk);
         if (n == 0) continue;
@@ -251,12 +256,39 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
             items[atomicAdd(&s_off[bucket(tiles)], 1)] = make_int4(s, kvh, a.t_offset, ctx);
             continue;
         }
+        const int li = atomicAdd(&s_nsplit, 1);
+        if (li < kPlanSplitList) {
+            s_split[li] = pr;
+            continue;
+        }
         const int ct = chunk * kTile;
         int pos = atomicAdd(&s_off[bucket(chunk)], n - 1);
         for (int j = 0; j < n - 1; ++j)
             items[pos + j] = make_int4(s, kvh | (j << 16), a.t_offset + j * ct, a.t_offset + (j + 1) * ct);
         pos = atomicAdd(&s_off[bucket(tiles - (n - 1) * chunk)], 1);
         items[pos] = make_int4(s, kvh | ((n - 1) << 16), a.t_offset + (n - 1) * ct, ctx);
+    }
+    __syncthreads();
+    // listed split pairs: one warp each, its lanes writing the splits (a long context has dozens)
+    const int lane = tid & 31;
+    const int nlisted = min(s_nsplit, kPlanSplitList);
+    for (int li = tid >> 5; li < nlisted; li += kPlanThreads / 32) {
+        const int pr = s_split[li];
+        const int s = pr / a.num_kv_heads, kvh = pr - s * a.num_kv_heads;
+        const int tiles = s < kPlanCache ? s_tiles[s] : dec_tiles(a, s, false);
+        const int n = dec_nsplit(tiles, whole, chunk);
+        const int ctx = s < kPlanCache ? s_ctx[s] : dec_ctx(a, s);
+        const int ct = chunk * kTile;
+        int pos = 0, last = 0;
+        if (lane == 0) {
+            pos = atomicAdd(&s_off[bucket(chunk)], n - 1);
+            last = atomicAdd(&s_off[bucket(tiles - (n - 1) * chunk)], 1);
+        }
+        pos = __shfl_sync(0xffffffffu, pos, 0);
+        last = __shfl_sync(0xffffffffu, last, 0);
+        for (int j = lane; j < n - 1; j += 32)
+            items[pos + j] = make_int4(s, kvh | (j << 16), a.t_offset + j * ct, a.t_offset + (j + 1) * ct);
+        if (lane == 0) items[last] = make_int4(s, kvh | ((n - 1) << 16), a.t_offset + (n - 1) * ct, ctx);
     }
 }
 
@@ -661,10 +693,12 @@ __global__ void __launch_bounds__(kThreads, 2)
 // Merge the per-split partials of one (sequence, q-head) by log-sum-exp.  kGroups x D threads: thread
 // (g, d) owns output element d for the partial slots g, g + kGroups, ...  The merge is a chain of dependent
 // reads, so it is kept short: the context length (an input of the call) is read before the wait for the
-// split kernel; after it, the planning header, the log-sum-exps and -- in the wide form, for the slot count
-// the host sized -- the first kPre partial elements of every thread are all requested at once, and the
-// slots past this pair's count are selected out afterwards.  The kGroups sums are added in shared memory.  A
-// pair that was not split returns at once (kGroups = 1 when no pair can have more than a few partials).
+// split kernel; after it, the planning header, the log-sum-exps and -- in the wide form (kGroups = 4, used
+// when few pairs have many partials: long contexts), for the slot count the host sized -- the first kPre
+// partial elements of every thread are all requested at once, and the slots past this pair's count are
+// selected out afterwards.  The narrow form requests its partials only once the header says the pair was
+// split: with many short CTAs, most of them for pairs that were not split, a request for nothing costs a
+// round trip to memory no call wrote in every wave of CTAs.  The kGroups sums are added in shared memory.
 constexpr int kLseCache = 1024;
 
 template <int D, int kGroups>
@@ -825,9 +859,9 @@ DecodePlan plan_decode(int32_t batch, int32_t num_kv_heads, int32_t max_context_
         chunk = ((int64_t)max_context_len + num_splits - 1) / num_splits;
         chunk = (chunk + kTile - 1) / kTile * kTile;
     } else {
-        // aim at about sixteen waves of two CTAs per SM over the whole batch, but
+        // aim at about eight waves of two CTAs per SM over the whole batch, but
         // never fewer than four tiles per CTA
-        const int64_t target = (int64_t)(num_sms > 0 ? num_sms : 148) * 2 * 16;
+        const int64_t target = (int64_t)(num_sms > 0 ? num_sms : 148) * 2 * 8;
         const int64_t pairs = (int64_t)batch * num_kv_heads;
         chunk = ((int64_t)max_context_len * pairs + target - 1) / target;
         chunk = (chunk + kTile - 1) / kTile * kTile;

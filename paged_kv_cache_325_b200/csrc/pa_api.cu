@@ -215,9 +215,10 @@ static pa_status decode_impl(void *out, const void *q, const void *k_cache, cons
 
     pa::DecodeArgs a = {};
     a.plan = pa::plan_decode(batch, num_kv_heads, max_context_len, num_splits, num_sms_current());
-    if (a.plan.max_splits > pa::kDecodeMaxSplits || num_kv_heads > pa::kDecodeMaxKvHeads)
-        return fail(PA_ERR_UNSUPPORTED, "more than %d context splits or %d KV heads", pa::kDecodeMaxSplits,
-                    pa::kDecodeMaxKvHeads);
+    if (a.plan.max_splits > pa::kDecodeMaxSplits || num_kv_heads > pa::kDecodeMaxKvHeads ||
+        (int64_t)batch * num_kv_heads > pa::kDecodeMaxPairs)
+        return fail(PA_ERR_UNSUPPORTED, "more than %d context splits, %d KV heads or %d (sequence, KV head) pairs",
+                    pa::kDecodeMaxSplits, pa::kDecodeMaxKvHeads, pa::kDecodeMaxPairs);
     const pa::DecodeWorkspace wl = pa::decode_workspace_layout(a.plan, batch, num_q_heads, num_kv_heads, head_dim);
     const size_t need = wl.total;
     if (!workspace || workspace_bytes < need)
@@ -313,7 +314,7 @@ pa_status pa_decode_split(void *out, const void *q, const void *k_cache, const v
 namespace {
 
 // Work split of the shared-prefix decode: the prefix keys are cut into chunks so that the prefix phase
-// has about two work units per SM; the private suffixes use the ordinary decode split.
+// has at most one work unit per SM; the private suffixes use the ordinary decode split.
 struct SharedPlan {
     pa::DecodePlan dplan;
     int32_t nchunks, key_chunk, ranks, slots;
@@ -327,7 +328,9 @@ SharedPlan plan_shared(int32_t batch, int32_t Hq, int32_t Hkv, int32_t D, int32_
     const int64_t nprefix = (int64_t)P * B;
     sp.ranks = (batch + 2 * TQ - 1) / (2 * TQ);
     const int64_t per_chunk_units = (int64_t)sp.ranks * Hkv;
-    int64_t nch = (2 * (int64_t)sms + per_chunk_units - 1) / per_chunk_units;
+    // at most one unit per SM: a unit of a few key tiles is mostly start-up, so a second round of units
+    // costs more than the longer chunks of a single round
+    int64_t nch = (int64_t)sms / per_chunk_units;
     const int64_t max_ch = (nprefix + 127) / 128;
     if (nch < 1) nch = 1;
     if (nch > max_ch) nch = max_ch;
@@ -443,9 +446,10 @@ pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
 
     // 2. private suffixes: split-KV decode from token nprefix on, partials after the prefix chunks;
     // 3. the combine kernel merges all partials of each (sequence, q-head)
-    if (sp.dplan.max_splits > pa::kDecodeMaxSplits || num_kv_heads > pa::kDecodeMaxKvHeads)
-        return fail(PA_ERR_UNSUPPORTED, "more than %d context splits or %d KV heads", pa::kDecodeMaxSplits,
-                    pa::kDecodeMaxKvHeads);
+    if (sp.dplan.max_splits > pa::kDecodeMaxSplits || num_kv_heads > pa::kDecodeMaxKvHeads ||
+        (int64_t)batch * num_kv_heads > pa::kDecodeMaxPairs)
+        return fail(PA_ERR_UNSUPPORTED, "more than %d context splits, %d KV heads or %d (sequence, KV head) pairs",
+                    pa::kDecodeMaxSplits, pa::kDecodeMaxKvHeads, pa::kDecodeMaxPairs);
     pa::DecodeArgs da = {};
     da.plan = sp.dplan;
     da.out = out;
@@ -653,9 +657,10 @@ pa_status pa_prefill_varlen_mixed(void *out, const void *q, int32_t total_q, con
     // 2. the decode rows (one new token, context n_k): the split-KV decode in its varlen mode
     pa::DecodeArgs da = {};
     da.plan = pa::plan_decode(batch, num_kv_heads, max_seqlen_k, 0, num_sms_current());
-    if (da.plan.max_splits > pa::kDecodeMaxSplits || num_kv_heads > pa::kDecodeMaxKvHeads)
-        return fail(PA_ERR_UNSUPPORTED, "more than %d context splits or %d KV heads", pa::kDecodeMaxSplits,
-                    pa::kDecodeMaxKvHeads);
+    if (da.plan.max_splits > pa::kDecodeMaxSplits || num_kv_heads > pa::kDecodeMaxKvHeads ||
+        (int64_t)batch * num_kv_heads > pa::kDecodeMaxPairs)
+        return fail(PA_ERR_UNSUPPORTED, "more than %d context splits, %d KV heads or %d (sequence, KV head) pairs",
+                    pa::kDecodeMaxSplits, pa::kDecodeMaxKvHeads, pa::kDecodeMaxPairs);
     const pa::DecodeWorkspace wl = pa::decode_workspace_layout(da.plan, batch, num_q_heads, num_kv_heads, head_dim);
     char *ws = static_cast<char *>(workspace) + pf_bytes;
     da.plan_ws = ws + wl.plan_off;

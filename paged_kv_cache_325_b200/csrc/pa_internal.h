@@ -44,6 +44,7 @@ DecodeWorkspace decode_workspace_layout(const DecodePlan &plan, int32_t batch, i
                                         int32_t num_kv_heads, int32_t head_dim, int32_t extra_slots = 0);
 constexpr int32_t kDecodeMaxSplits = 32767;     // split index and KV head share one int of an item
 constexpr int32_t kDecodeMaxKvHeads = 65535;
+constexpr int32_t kDecodeMaxPairs = 1 << 30;    // batch * num_kv_heads: the planning kernel counts pairs in int
 
 struct DecodeArgs {
     void *out;

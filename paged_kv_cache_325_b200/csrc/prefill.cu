@@ -805,15 +805,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int q = 0; q < 4; ++q) tmem_ld32(lane_base + col_s(x) + q * 32, sr[q]);
                 tc_wait_ld();
                 const int thr = lim - (U.kbeg + j * kN);   // keys e <= thr are visible
-                // row maximum: three-input max over pairs, eight independent chains
-                float mx[8];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) mx[c] = -INFINITY;
+                // row maximum: three-input max over pairs, four independent chains
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 if (thr >= kN - 1) {
 #pragma unroll
-                    for (int e = 0; e < kN; e += 16)
+                    for (int e = 0; e < kN; e += 8)
 #pragma unroll
-                        for (int c = 0; c < 8; ++c)
+                        for (int c = 0; c < 4; ++c)
                             mx[c] = max3f(mx[c], __uint_as_float(sr[(e + 2 * c) >> 5][(e + 2 * c) & 31]),
                                           __uint_as_float(sr[(e + 2 * c + 1) >> 5][(e + 2 * c + 1) & 31]));
                 } else {
@@ -821,11 +819,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < kN; ++e) {
                         const float v = e <= thr ? __uint_as_float(sr[e >> 5][e & 31]) : -INFINITY;
                         sr[e >> 5][e & 31] = __float_as_uint(v);
-                        mx[e & 7] = fmaxf(mx[e & 7], v);
+                        mx[e & 3] = fmaxf(mx[e & 3], v);
                     }
                 }
-                const float m_new =
-                    fmaxf(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], max3f(mx[5], mx[6], mx[7]))) * sl;
+                const float m_new = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl;
                 float corr = 1.f;
                 bool rescale = false;
                 if (m_new > m_ref + 8.f) {                  // also true while m_ref is -inf

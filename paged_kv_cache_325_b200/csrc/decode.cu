@@ -250,6 +250,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         const int s = pr / a.num_kv_heads, kvh = pr - s * a.num_kv_heads;
         const int tiles = s < kPlanCache ? s_tiles[s] : dec_tiles(a, s, false);
         const int n = dec_nsplit(tiles, whole, chunk);
+        if (a.merge_count) a.merge_count[pr] = n;    // splits of the pair still to finish (the decode counts down)
         if (n == 0) continue;
         const int ctx = s < kPlanCache ? s_ctx[s] : dec_ctx(a, s);
         if (n == 1) {
@@ -296,6 +297,11 @@ struct DecItem {
     int s, kvh, split, t_begin, t_end, ntiles, ctx;
 };
 
+// In-kernel merge of a split pair: weights of up to kMergeW (head, split) partials staged in shared memory;
+// used when the host plan cuts a pair into at most kMergeMaxSplits splits.
+constexpr int kMergeW = 1024;
+constexpr int kMergeMaxSplits = 8;
+
 // A consumer-wide vote (the 128 threads of warps 0-3, named barrier 1): true iff v is true for all.
 __device__ __forceinline__ bool consumers_all(bool v) {
     uint32_t r;
@@ -306,6 +312,92 @@ __device__ __forceinline__ bool consumers_all(bool v) {
         : "r"((uint32_t)v), "n"(kConsumerWarps * 32)
         : "memory");
     return r != 0;
+}
+
+// Merge the nsp partials of (sequence s, KV head kvh) -- every split of the pair -- into its G output rows:
+// log-sum-exp weights staged in shared memory, then weighted sums of the fp32 partials, four elements per
+// thread.  Run by the 128 consumer threads of the CTA that finished the pair's last split; red_o (the merge
+// area) is free.
+template <int D>
+__device__ __forceinline__ void merge_pair(const DecodeArgs &a, int s, int kvh, int nsp, int G, float *red_o,
+                                           float *s_w, float *s_wsum) {
+    __threadfence();   // (thread 0 acquired the other splits' partials; order this thread's reads after it)
+    const int tid = threadIdx.x;
+    const int64_t pb0 = ((int64_t)s * a.num_q_heads + (int64_t)kvh * G) * a.part_slots;
+    const int64_t orow = dec_row(a, s) * a.num_q_heads + (int64_t)kvh * G;
+    if (G * nsp <= kMergeW) {
+        // weights exp2(lse_j - max) per head, staged in shared memory, and their sums
+        for (int i = tid; i < G * nsp; i += kConsumerWarps * 32) {
+            const int g = i / nsp, j = i - g * nsp;
+            s_w[i] = __ldcg(a.part_lse + pb0 + (int64_t)g * a.part_slots + j);
+        }
+        consumer_sync();
+        if (tid < G) {
+            float m = -INFINITY, sum = 0.f;
+            for (int j = 0; j < nsp; ++j) m = fmaxf(m, s_w[tid * nsp + j]);
+            for (int j = 0; j < nsp; ++j) {
+                const float w = fast_exp2(s_w[tid * nsp + j] - m);
+                s_w[tid * nsp + j] = w;
+                sum += w;
+            }
+            s_wsum[tid] = sum;
+        }
+        consumer_sync();
+        // weighted sums over the splits, four elements per thread; with few columns several threads
+        // share a column (each a stride of the splits) and their sums meet in the merge area
+        const int ncol = G * D / 4;
+        const int ngrp = max(1, min(4, kConsumerWarps * 32 / ncol));
+        float4 *acc = reinterpret_cast<float4 *>(red_o);   // [ngrp][ncol]
+        for (int c = tid; c < ncol * ngrp; c += kConsumerWarps * 32) {
+            const int col = c % ncol, grp = c / ncol;
+            const int g = col / (D / 4), d4 = col % (D / 4);
+            const float4 *src = reinterpret_cast<const float4 *>(a.part_o + (pb0 + (int64_t)g * a.part_slots) * D) + d4;
+            float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+            for (int j = grp; j < nsp; j += ngrp) {
+                const float w = s_w[g * nsp + j];
+                const float4 v = __ldcg(src + (int64_t)j * (D / 4));
+                t.x += w * v.x;
+                t.y += w * v.y;
+                t.z += w * v.z;
+                t.w += w * v.w;
+            }
+            acc[grp * ncol + col] = t;
+        }
+        consumer_sync();
+        for (int col = tid; col < ncol; col += kConsumerWarps * 32) {
+            float4 t = acc[col];
+            for (int grp = 1; grp < ngrp; ++grp) {
+                const float4 u = acc[grp * ncol + col];
+                t.x += u.x;
+                t.y += u.y;
+                t.z += u.z;
+                t.w += u.w;
+            }
+            const int g = col / (D / 4), d4 = col % (D / 4);
+            const float inv = 1.f / s_wsum[g];
+            uint2 o2;
+            o2.x = pack_bf16(t.x * inv, t.y * inv);
+            o2.y = pack_bf16(t.z * inv, t.w * inv);
+            reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.out) + (orow + g) * D)[d4] = o2;
+        }
+    } else {
+        // more (head, split) partials than the staging area holds (a very long context cut into
+        // thousands of splits): element by element
+        for (int e = tid; e < G * D; e += kConsumerWarps * 32) {
+            const int g = e / D, d = e % D;
+            const int64_t pb = pb0 + (int64_t)g * a.part_slots;
+            float mt = -INFINITY;
+            for (int j = 0; j < nsp; ++j) mt = fmaxf(mt, __ldcg(a.part_lse + pb + j));
+            float num = 0.f, den = 0.f;
+            for (int j = 0; j < nsp; ++j) {
+                const float w = fast_exp2(__ldcg(a.part_lse + pb + j) - mt);
+                num += w * __ldcg(a.part_o + (pb + j) * D + d);
+                den += w;
+            }
+            static_cast<__nv_bfloat16 *>(a.out)[(orow + g) * D + d] = __float2bfloat16_rn(num / den);
+        }
+    }
 }
 
 // kFused: the pa_store_kv_decode variant (store fused in); a separate instantiation, so the plain decode
@@ -441,6 +533,32 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: matrix index / row this lane addresses
     uint32_t gt = 0, nqi = 0;
     bool ok = true;
+    // In-kernel merge (a.merge_count): thread 0 counts a finished split down with an atomic whose result it
+    // looks at only one item later (or when the stream ends), so no consumer waits for the round trip; if the
+    // count reached zero this CTA finished the pair's last split and merges the pair (flush_pending).
+    int pend_left = 0, hdr_whole = -1, hdr_chunk = 0;
+    int4 pend = make_int4(0, 0, 0, 0);   // s, kvh, ctx, counted
+    __shared__ int4 s_pend;
+    __shared__ float s_w[kMergeW], s_wsum[16];
+    auto flush_pending = [&]() {
+        if (threadIdx.x == 0) {
+            int nsp = 0;
+            if (pend.w && pend_left == 1) {
+                if (hdr_whole < 0) {
+                    const DecPlanHdr *hdr = reinterpret_cast<const DecPlanHdr *>(a.plan_ws);
+                    hdr_whole = __ldcg(&hdr->whole);
+                    hdr_chunk = __ldcg(&hdr->chunk);
+                }
+                nsp = dec_nsplit((pend.z - a.t_offset + kTile - 1) / kTile, hdr_whole, hdr_chunk);
+            }
+            s_pend = make_int4(pend.x, pend.y, nsp, 0);
+            pend.w = 0;
+        }
+        consumer_sync();
+        const int4 pm = s_pend;
+        if (pm.z > 0) merge_pair<D>(a, pm.x, pm.y, pm.z, G, red_o, s_w, s_wsum);
+        consumer_sync();   // s_pend and the merge area are free again
+    };
     for (;;) {
         // the next item, from the producer; the consumers leave together at the end marker or after a
         // timed-out wait (a wait that gave up leaves the results garbage and dev_error says so)
@@ -686,8 +804,21 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (d == 0) a.part_lse[pi] = mt + __log2f(lt);
             }
         }
+        if (a.merge_count) {
+            flush_pending();   // the split counted down one item ago (its atomic has long returned)
+            if (!direct) {
+                // this split is finished: count it down (release: every consumer's partial stores, ordered
+                // before thread 0 by the barrier, are visible before the count; acquire for the last one,
+                // which merges)
+                if (threadIdx.x == 0) {
+                    pend_left = atomic_add_acq_rel(a.merge_count + (int64_t)it.s * a.num_kv_heads + it.kvh, -1);
+                    pend = make_int4(it.s, it.kvh, it.ctx, 1);
+                }
+            }
+        }
         consumer_sync();   // the merge area is free for the next item
     }
+    if (a.merge_count) flush_pending();   // the last split this CTA counted down
 }
 
 // Merge the per-split partials of one (sequence, q-head) by log-sum-exp.  kGroups x D threads: thread
@@ -819,7 +950,7 @@ cudaError_t launch_decode_d(const DecodeArgs &a, const CUtensorMap &tm_k, const 
 
     // 1. the item table; 2. the persistent decode, launched as its programmatic dependent so that its
     // set-up overlaps the planning (its producer waits for the table with griddepcontrol.wait);
-    // 3. the combine, for pairs that were split
+    // 3. the combine, only when partials come from elsewhere too (the split kernel merges its own)
     decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(a, grid);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -834,7 +965,7 @@ cudaError_t launch_decode_d(const DecodeArgs &a, const CUtensorMap &tm_k, const 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kernel, tm_k, tm_v, a);
-    if (e != cudaSuccess || (a.plan.max_splits == 1 && a.part_base == 0)) return e;
+    if (e != cudaSuccess || (a.plan.max_splits == 1 && a.part_base == 0) || a.merge_count) return e;
 
     // a few partials per pair, or so many pairs that four threads per element would not fit the GPU at
     // once (a large batch): one thread per element; many partials for few pairs (long contexts): four
@@ -876,9 +1007,15 @@ DecodePlan plan_decode(int32_t batch, int32_t num_kv_heads, int32_t max_context_
     return p;
 }
 
-size_t decode_plan_bytes(const DecodePlan &plan, int32_t batch, int32_t num_kv_heads) {
+// Planning area: header, item table, then one merge counter per (sequence, KV head).
+static size_t decode_counter_offset(const DecodePlan &plan, int32_t batch, int32_t num_kv_heads) {
     const size_t items = (size_t)batch * num_kv_heads * (plan.max_splits > 0 ? plan.max_splits : 1);
-    return (kPlanHdrBytes + items * sizeof(int4) + 255) / 256 * 256;
+    return kPlanHdrBytes + items * sizeof(int4);
+}
+
+size_t decode_plan_bytes(const DecodePlan &plan, int32_t batch, int32_t num_kv_heads) {
+    const size_t counters = (size_t)batch * num_kv_heads * sizeof(int32_t);
+    return (decode_counter_offset(plan, batch, num_kv_heads) + counters + 255) / 256 * 256;
 }
 
 DecodeWorkspace decode_workspace_layout(const DecodePlan &plan, int32_t batch, int32_t num_q_heads,
@@ -894,8 +1031,18 @@ DecodeWorkspace decode_workspace_layout(const DecodePlan &plan, int32_t batch, i
     return w;
 }
 
-cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+cudaError_t launch_decode(const DecodeArgs &args, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                           cudaStream_t stream) {
+    DecodeArgs a = args;
+    // Split pairs are merged in the split kernel when a pair has only a few splits and no partials come from
+    // elsewhere: that saves the combine launch, and each merge is short.  With many splits per pair (long
+    // contexts) the pairs' last splits finish together at the end of the grid, and a CTA per pair merging
+    // dozens of partials makes a longer tail than the combine kernel, which spreads the merge over many
+    // CTAs (measured: 4 splits per pair, -2 us; 32, +10 us).
+    a.merge_count = a.part_base == 0 && a.plan.max_splits > 1 && a.plan.max_splits <= kMergeMaxSplits
+                        ? reinterpret_cast<int32_t *>(static_cast<char *>(a.plan_ws) +
+                                                      decode_counter_offset(a.plan, a.batch, a.num_kv_heads))
+                        : nullptr;
     if (a.head_dim == 128) return launch_decode_d<128>(a, tm_k, tm_v, stream);
     return launch_decode_d<64>(a, tm_k, tm_v, stream);
 }

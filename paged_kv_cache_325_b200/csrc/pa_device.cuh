@@ -76,6 +76,13 @@ PA_DEVICE bool mbar_test_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Atomic add at GPU scope with acquire-release ordering; returns the old value.
+PA_DEVICE int32_t atomic_add_acq_rel(int32_t *p, int32_t v) {
+    int32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 PA_DEVICE uint64_t global_timer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

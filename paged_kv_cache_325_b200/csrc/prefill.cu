@@ -18,9 +18,11 @@
 //    head); a one-CTA planning kernel writes the units into a table ordered by
 //    decreasing cost (last tiles of every sequence first), and persistent CTAs,
 //    one per SM, take them with an atomic counter;
-//  * warp 8 (TMA): per unit, both Q tiles (3-D tensor map over q), then the
-//    K and V tiles of 128 keys, gathered block by block through block_table,
-//    into a ring of shared-memory slots guarded by mbarriers;
+//  * warp 11 (Q): per unit, both Q tiles (3-D tensor map over q) into the Q
+//    buffer once the previous unit's S products have read it; warp 8 (K/V):
+//    the K and V tiles of 128 keys, gathered block by block through
+//    block_table, into a ring of shared-memory slots guarded by mbarriers,
+//    running ahead into the next units so that a unit starts on loaded tiles;
 //  * warp 9 (MMA): one thread issues tcgen05.mma.cta_group::1.kind::f16 in the
 //    order S_A(0) S_B(0) | PV_A(j) S_A(j+1) PV_B(j) S_B(j+1) | ..., so the
 //    tensor cores work on one tile while the other tile's softmax runs.
@@ -51,8 +53,10 @@ constexpr int kN = 128;                // keys per K/V tile
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kFixWarp = 10;
-constexpr int kThreads = 384;          // 2 softmax warpgroups + TMA warp + MMA warp + V-fix warp + warp 11, which
-                                       // has no role: it completes the third warpgroup for the register split
+constexpr int kQWarp = 11;
+constexpr int kThreads = 384;          // 2 softmax warpgroups + K/V TMA warp + MMA warp + V-fix warp + Q TMA warp
+constexpr int kVlast = 4;              // ring of last-V barriers: the K/V loads may run this many units ahead of
+                                       // the V-fix warp
 // Register split (setmaxnreg): a 384-thread block is launched with kRegsAtLaunch registers per thread (the
 // most that ptxas gives it); the third warpgroup (TMA, MMA, V-fix, spare) drops to kRegsOther and the two
 // softmax warpgroups, which hold a 128-column S row and a 128-column O row per thread, rise to kRegsSoftmax.
@@ -65,6 +69,13 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsAtLau
 constexpr int kRowBytes = 128;         // one 64-element bf16 swizzle row
 constexpr int kSlab = kM * kRowBytes;  // 128 rows x 128 B = 16 KB
 constexpr int kUnitQueue = 4;          // unit ids handed from the TMA warp to the other roles
+// Ring of "last V tile fixed" barriers, one entry per unit in turn.  The V-fix warp may run ahead of the MMA
+// thread, but by fewer than kFixRing units: it fixes unit m only after the K/V warp pushed m to the unit queue,
+// which needs every consumer, the MMA thread included, to have popped unit m - kUnitQueue; the MMA thread pops
+// a unit only after finishing the one before, so it has waited for the fix of unit m - kUnitQueue - 1 and
+// earlier.  Entry m % kFixRing is therefore never two phases ahead of its waiter.
+constexpr int kFixRing = 2 * kUnitQueue;
+static_assert(kFixRing > kUnitQueue + 1, "fix ring deeper than the unit queue's lead");
 constexpr int kPlanThreads = 1024;
 
 // kFused: the store fused in (pa_store_kv_prefill_varlen) needs a staging area for the rows it copies; at
@@ -81,8 +92,8 @@ struct PrefillCfg {
     static constexpr int kStageBytes = kFused ? kStageTokens * 4 * D : 0;
     static constexpr int kBarOff = kStageOff + kStageBytes;
     // kv_full[S] kv_empty[S] q_full q_empty s_full[2] p_full[2] o_full[2] o_empty[2] done uq_full[4] uq_empty[4]
-    // v_fixed vlast_full[2] cp_full
-    static constexpr int kNumBars = 2 * kSlots + 11 + 2 * kUnitQueue + 3 + 1;
+    // v_fixed[kFixRing] vlast_full[kVlast] vlast_empty[kVlast] cp_full
+    static constexpr int kNumBars = 2 * kSlots + 11 + 2 * kUnitQueue + kFixRing + 2 * kVlast + 1;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 64 + kUnitQueue * 64 + 1024;
     static constexpr uint32_t kTmemCols = 512;                  // S_A 0, O_A 128, S_B 256, O_B 384
                                                                 // (P_X, bf16, overwrites the first 64 columns of S_X)
@@ -304,12 +315,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *done = o_empty + 2;
     uint64_t *uq_full = done + 1;      // [kUnitQueue]
     uint64_t *uq_empty = uq_full + kUnitQueue;
-    uint64_t *v_fixed = uq_empty + kUnitQueue;   // the last V tile of a unit is ready for PV
-    // The last V tile of a unit lands on its own barrier, alternating by unit: the TMA warp runs at most
-    // one unit ahead of the V-fix warp (the next unit's loads wait for this unit's S products, and those
-    // wait for the fix), so two barriers keep every phase distinct.
-    uint64_t *vlast_full = v_fixed + 1;           // [2]
-    uint64_t *cp_full = vlast_full + 2;           // fused store: a copy round's rows are in the staging area
+    uint64_t *v_fixed = uq_empty + kUnitQueue;   // [kFixRing] the last V tile of a unit is ready for PV
+    // The last V tile of a unit lands on its own barrier, from a ring of kVlast taken in unit order: the V-fix
+    // warp arrives on the matching vlast_empty once it has waited, and the K/V warp waits for that before it
+    // reuses the entry, so every phase is waited for in order whatever the K/V warp's lead.
+    uint64_t *vlast_full = v_fixed + kFixRing;    // [kVlast]
+    uint64_t *vlast_empty = vlast_full + kVlast;  // [kVlast]
+    uint64_t *cp_full = vlast_empty + kVlast;     // fused store: a copy round's rows are in the staging area
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
     // set by the first wait of this CTA that gives up; every other wait then gives up at once
     volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
@@ -341,13 +353,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(o_empty + x), 4);
         }
         mbar_init(smem_u32(done), 1);
-        mbar_init(smem_u32(v_fixed), 1);
-        mbar_init(smem_u32(vlast_full), 1);
-        mbar_init(smem_u32(vlast_full + 1), 1);
+        for (int i = 0; i < kFixRing; ++i) mbar_init(smem_u32(v_fixed + i), 1);
+        for (int i = 0; i < kVlast; ++i) {
+            mbar_init(smem_u32(vlast_full + i), 1);
+            mbar_init(smem_u32(vlast_empty + i), 1);
+        }
         mbar_init(smem_u32(cp_full), 1);
         for (int i = 0; i < kUnitQueue; ++i) {
             mbar_init(smem_u32(uq_full + i), 1);
-            mbar_init(smem_u32(uq_empty + i), 10);  // the MMA warp, the V-fix warp, the eight softmax warps
+            mbar_init(smem_u32(uq_empty + i), 11);  // the MMA, V-fix and Q warps, the eight softmax warps
         }
         fence_barrier_init();
     }
@@ -406,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int4 rec = units[u];
                 return unit_from_record(a, rec, geo[rec.x], TQ);
             };
-            uint32_t nq = 0, L = 0, nvlast = 0;
+            uint32_t L = 0, nvlast = 0;
             bool ok = true;
             Unit next = decode(fetch());
             for (uint32_t nu = 0;; ++nu) {
@@ -427,31 +441,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // take the next unit now; its id and record loads overlap this unit's copies
                 const int next_u = fetch();
                 if (U.valid) {
-                    // Q first: the wait for the Q buffer (free once the previous unit's S products complete,
-                    // which the MMA thread issues only after the V fix of the unit before it) keeps this warp at
-                    // most one unit ahead of the V-fix warp, which the two alternating last-V barriers rely on.
+                    // K and V only (the Q warp loads Q): this warp runs ahead into the next units as far as the
+                    // ring slots, the unit queue and the last-V ring let it, so a unit's first tiles are loaded
+                    // while the previous unit still computes
                     const int32_t *bt = a.block_table + (int64_t)U.s * a.bt_stride;
                     const int kend = max(U.kend[0], U.kend[1]);
                     int chunk = -32, ids = 0;            // block_table[chunk + lane] lives in `ids` of that lane
                     if (ok && U.nk > 0) ++nvlast;
-                    const int nloads = 2 * U.nk, pre = 0;
-                    for (int li = 0; li <= nloads && ok; ++li) {
-                        if (li == pre) {
-                            if (nq > 0 && !mbar_wait(smem_u32(q_empty), (nq - 1) & 1, a.dev_error, 0xffffffffu, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            if (lane == 0) {
-                                mbar_arrive_expect_tx(smem_u32(q_full), (uint32_t)(2 * C::kTileBytes));
-                                for (int x = 0; x < 2; ++x)
-#pragma unroll
-                                    for (int h = 0; h < C::kHalves; ++h)
-                                        tma_load_3d(q_s + x * C::kTileBytes + h * kSlab, &tm_q, h * 64, U.kvh * G,
-                                                    U.q0 + U.tok0[x], smem_u32(q_full));
-                            }
-                            ++nq;
-                        }
-                        if (li == nloads) break;
+                    const int nloads = 2 * U.nk;
+                    for (int li = 0; li < nloads && ok; ++li) {
                         const int j = li >> 1, kv = li & 1;
                         const int key0 = U.kbeg + j * kN;
                         const int nbox = (min(kN, kend - key0) + box - 1) / box;
@@ -469,7 +467,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // the last V tile of the unit lands on its own barrier (the V-fix warp consumes it in
                         // order); the ring slot's barrier still completes one phase, with no bytes
                         const bool vlast = kv == 1 && j == U.nk - 1;
-                        const uint32_t fb = smem_u32(vlast ? vlast_full + ((nvlast - 1) & 1) : kv_full + slot2);
+                        if (vlast && nvlast > (uint32_t)kVlast &&
+                            !mbar_wait(smem_u32(vlast_empty + (nvlast - 1) % kVlast), ((nvlast - 1) / kVlast - 1) & 1,
+                                       a.dev_error, 0xffffffffu, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t fb = smem_u32(vlast ? vlast_full + (nvlast - 1) % kVlast : kv_full + slot2);
                         if (lane == 0) {
                             if (vlast) mbar_arrive(smem_u32(kv_full + slot2));
                             mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * kRowBytes * C::kHalves));
@@ -506,14 +510,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 next = decode(next_u);
             }
-            // Leave no TMA copy in flight: wait (bounded) for the last load of every ring slot and for the
-            // last Q load.  On the normal path the MMA warp consumed them all and these return at once; they
-            // ignore the abort flag, since the copies land in this CTA's shared memory whatever happened.
+            // Leave no TMA copy in flight: wait (bounded) for the last load of every ring slot and of every
+            // last-V barrier.  On the normal path the MMA and V-fix warps consumed them all and these return at
+            // once; they ignore the abort flag, since the copies land in this CTA's shared memory whatever
+            // happened.
             for (uint32_t i = (L > (uint32_t)C::kSlots ? L - C::kSlots : 0); i < L; ++i)
                 mbar_wait(smem_u32(kv_full + i % C::kSlots), (i / C::kSlots) & 1, a.dev_error);
+            for (uint32_t i = (nvlast > (uint32_t)kVlast ? nvlast - kVlast : 0); i < nvlast; ++i)
+                mbar_wait(smem_u32(vlast_full + i % kVlast), (i / kVlast) & 1, a.dev_error);
+        } else if (warp == kQWarp) {
+            // ============================================================== Q ==
+            // Both Q tiles of each unit, as soon as the previous unit's S products have read the buffer.
+            if (lane == 0) tma_prefetch_desc(&tm_q);
+            uint32_t nq = 0;
+            for (uint32_t k = 0;; ++k) {
+                Unit U;
+                if (!pop_unit(k, lane == 0, U)) break;
+                if (!U.valid) continue;
+                if (nq > 0 && !mbar_wait(smem_u32(q_empty), (nq - 1) & 1, a.dev_error, 0xffffffffu, abort_flag)) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(smem_u32(q_full), (uint32_t)(2 * C::kTileBytes));
+                    for (int x = 0; x < 2; ++x)
+#pragma unroll
+                        for (int h = 0; h < C::kHalves; ++h)
+                            tma_load_3d(q_s + x * C::kTileBytes + h * kSlab, &tm_q, h * 64, U.kvh * G, U.q0 + U.tok0[x],
+                                        smem_u32(q_full));
+                }
+                __syncwarp();
+                ++nq;
+            }
+            // the last Q load has landed before the CTA can exit (bounded; ignores the abort flag)
             if (nq > 0) mbar_wait(smem_u32(q_full), (nq - 1) & 1, a.dev_error);
-            for (uint32_t i = (nvlast > 2 ? nvlast - 2 : 0); i < nvlast; ++i)
-                mbar_wait(smem_u32(vlast_full + (i & 1)), (i >> 1) & 1, a.dev_error);
         } else if (warp == kMmaWarp) {
             // ============================================================ MMA ==
             // One thread: the tensor cores keep almost no queue, so this thread does nothing but wait for
@@ -578,7 +605,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t vidx = L + 2 * j + 1, knext = L + 2 * j + 2;
                         if (j == U.nk - 1) {
                             // the V-fix warp has zeroed the rows past the key range of the unit's last V tile
-                            if (!mbar_wait(smem_u32(v_fixed), nfix & 1, a.dev_error, 0xffffffffu, abort_flag)) { ok = false; break; }
+                            if (!mbar_wait(smem_u32(v_fixed + nfix % kFixRing), (nfix / kFixRing) & 1, a.dev_error,
+                                           0xffffffffu, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
                             ++nfix;
                         } else if (!wait_slot(vidx)) {
                             ok = false;
@@ -704,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 U.valid = 0;
                 if (more && !pop_unit(k, lane == 0, U)) more = false;
                 if (more && !U.valid) continue;
-                const uint32_t vbar = smem_u32(vlast_full + (nfx & 1)), vpar = (nfx >> 1) & 1;
+                const uint32_t vbar = smem_u32(vlast_full + nfx % kVlast), vpar = (nfx / kVlast) & 1;
                 if (kFused) {
                     // pump the copy engine until the unit's last V tile lands (a fix first, always) or, with
                     // no unit left, until nothing is pending; leave room in the FIFO for this unit.  Bounded:
@@ -740,6 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t vidx = L + 2 * (U.nk - 1) + 1;
                 L += 2 * U.nk;
                 if (!mbar_wait(vbar, vpar, a.dev_error, 0xffffffffu, abort_flag)) break;
+                if (lane == 0) mbar_arrive(smem_u32(vlast_empty + nfx % kVlast));   // the entry may be reused
                 ++nfx;
                 const int valid = max(U.kend[0], U.kend[1]) - (U.kbeg + (U.nk - 1) * kN);
                 if (valid < kN) {
@@ -754,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     fence_proxy_async_smem();
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(v_fixed));
+                if (lane == 0) mbar_arrive(smem_u32(v_fixed + (nfx - 1) % kFixRing));
                 if (kFused && U.chunk == 0) {
                     // this unit's own tokens: tile A's, then tile B's (present only when tile A is full); the
                     // loop above left room in the FIFO

@@ -122,10 +122,44 @@ __device__ __forceinline__ int dec_tiles(const DecodeArgs &a, int s, bool report
     return (ctx - a.t_offset + kTile - 1) / kTile;
 }
 
-// Splits of a pair with `tiles` tiles under (whole, chunk); 0 tiles: no item.
+// How a pair of `tiles` tiles is cut under (whole, chunk).  At most `whole` tiles: one item.  Longer: pieces of
+// `chunk` tiles, except that the last two chunks' worth (the remainder included) is cut into kTailPieces
+// smaller pieces, so that the items handed out last -- the shortest, in the longest-first order -- are small
+// and the CTAs finish together.  whole == 0 (a split count the caller fixed): uniform pieces of `chunk`.
+constexpr int kTailPieces = 4;
+struct SplitGeom {
+    int n;       // splits
+    int nfull;   // leading splits of `chunk` tiles
+    int np;      // tail pieces after them: `base` tiles, the first `extra` of them one more
+    int base, extra;
+};
+__device__ __forceinline__ SplitGeom dec_split_geom(int tiles, int whole, int chunk) {
+    SplitGeom g;
+    g.n = g.nfull = g.np = g.base = g.extra = 0;
+    if (tiles == 0) return g;
+    if (tiles <= whole) {
+        g.n = 1;
+        g.np = 1;
+        g.base = tiles;
+        return g;
+    }
+    const int n = (tiles + chunk - 1) / chunk;
+    g.nfull = whole == 0 || n < 2 ? n - 1 : n - 2;
+    const int tail = tiles - g.nfull * chunk;
+    g.np = whole == 0 || n < 2 ? 1 : min(kTailPieces, tail);
+    g.base = tail / g.np;
+    g.extra = tail - g.base * g.np;
+    g.n = g.nfull + g.np;
+    return g;
+}
 __device__ __forceinline__ int dec_nsplit(int tiles, int whole, int chunk) {
-    if (tiles == 0) return 0;
-    return tiles <= whole ? 1 : (tiles + chunk - 1) / chunk;
+    return dec_split_geom(tiles, whole, chunk).n;
+}
+// First tile of split j (j == n: the end).
+__device__ __forceinline__ int dec_split_begin(const SplitGeom &g, int chunk, int j) {
+    if (j <= g.nfull) return j * chunk;
+    const int k = j - g.nfull;
+    return g.nfull * chunk + k * g.base + min(k, g.extra);
 }
 
 __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeArgs a, int32_t num_ctas) {
@@ -173,14 +207,11 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     auto bucket = [](int tiles) { return min(tiles, kPlanBuckets - 1); };
     for (int s = tid; s < a.batch; s += kPlanThreads) {
         const int tiles = s < kPlanCache ? s_tiles[s] : dec_tiles(a, s, false);
-        const int n = dec_nsplit(tiles, whole, chunk);
-        if (n == 0) continue;
-        if (n == 1) {
-            atomicAdd(&s_off[bucket(tiles)], a.num_kv_heads);
-        } else {
-            atomicAdd(&s_off[bucket(chunk)], (n - 1) * a.num_kv_heads);
-            atomicAdd(&s_off[bucket(tiles - (n - 1) * chunk)], a.num_kv_heads);
-        }
+        const SplitGeom g = dec_split_geom(tiles, whole, chunk);
+        if (g.n == 0) continue;
+        if (g.nfull > 0) atomicAdd(&s_off[bucket(chunk)], g.nfull * a.num_kv_heads);
+        if (g.extra > 0) atomicAdd(&s_off[bucket(g.base + 1)], g.extra * a.num_kv_heads);
+        atomicAdd(&s_off[bucket(g.base)], (g.np - g.extra) * a.num_kv_heads);
     }
     __syncthreads();
     {   // exclusive scan over the buckets from the longest down: thread t owns bucket kPlanBuckets - 1 - t
@@ -249,11 +280,11 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     for (int pr = tid; pr < npairs; pr += kPlanThreads) {
         const int s = pr / a.num_kv_heads, kvh = pr - s * a.num_kv_heads;
         const int tiles = s < kPlanCache ? s_tiles[s] : dec_tiles(a, s, false);
-        const int n = dec_nsplit(tiles, whole, chunk);
-        if (a.merge_count) a.merge_count[pr] = n;    // splits of the pair still to finish (the decode counts down)
-        if (n == 0) continue;
+        const SplitGeom g = dec_split_geom(tiles, whole, chunk);
+        if (a.merge_count) a.merge_count[pr] = g.n;   // splits of the pair still to finish (the decode counts down)
+        if (g.n == 0) continue;
         const int ctx = s < kPlanCache ? s_ctx[s] : dec_ctx(a, s);
-        if (n == 1) {
+        if (g.n == 1) {
             items[atomicAdd(&s_off[bucket(tiles)], 1)] = make_int4(s, kvh, a.t_offset, ctx);
             continue;
         }
@@ -262,12 +293,12 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
             s_split[li] = pr;
             continue;
         }
-        const int ct = chunk * kTile;
-        int pos = atomicAdd(&s_off[bucket(chunk)], n - 1);
-        for (int j = 0; j < n - 1; ++j)
-            items[pos + j] = make_int4(s, kvh | (j << 16), a.t_offset + j * ct, a.t_offset + (j + 1) * ct);
-        pos = atomicAdd(&s_off[bucket(tiles - (n - 1) * chunk)], 1);
-        items[pos] = make_int4(s, kvh | ((n - 1) << 16), a.t_offset + (n - 1) * ct, ctx);
+        // past the list's capacity: this thread writes the pair's splits, one slot each
+        for (int j = 0; j < g.n; ++j) {
+            const int b0 = dec_split_begin(g, chunk, j), b1 = dec_split_begin(g, chunk, j + 1);
+            items[atomicAdd(&s_off[bucket(b1 - b0)], 1)] =
+                make_int4(s, kvh | (j << 16), a.t_offset + b0 * kTile, j == g.n - 1 ? ctx : a.t_offset + b1 * kTile);
+        }
     }
     __syncthreads();
     // listed split pairs: one warp each, its lanes writing the splits (a long context has dozens)
@@ -277,19 +308,22 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         const int pr = s_split[li];
         const int s = pr / a.num_kv_heads, kvh = pr - s * a.num_kv_heads;
         const int tiles = s < kPlanCache ? s_tiles[s] : dec_tiles(a, s, false);
-        const int n = dec_nsplit(tiles, whole, chunk);
+        const SplitGeom g = dec_split_geom(tiles, whole, chunk);
         const int ctx = s < kPlanCache ? s_ctx[s] : dec_ctx(a, s);
         const int ct = chunk * kTile;
-        int pos = 0, last = 0;
-        if (lane == 0) {
-            pos = atomicAdd(&s_off[bucket(chunk)], n - 1);
-            last = atomicAdd(&s_off[bucket(tiles - (n - 1) * chunk)], 1);
-        }
+        // the full chunks take consecutive slots of their bucket (lane 0 reserves them); each tail piece
+        // (lanes 0 .. np-1) reserves its own slot
+        int pos = 0;
+        if (lane == 0 && g.nfull > 0) pos = atomicAdd(&s_off[bucket(chunk)], g.nfull);
         pos = __shfl_sync(0xffffffffu, pos, 0);
-        last = __shfl_sync(0xffffffffu, last, 0);
-        for (int j = lane; j < n - 1; j += 32)
+        for (int j = lane; j < g.nfull; j += 32)
             items[pos + j] = make_int4(s, kvh | (j << 16), a.t_offset + j * ct, a.t_offset + (j + 1) * ct);
-        if (lane == 0) items[last] = make_int4(s, kvh | ((n - 1) << 16), a.t_offset + (n - 1) * ct, ctx);
+        if (lane < g.np) {
+            const int j = g.nfull + lane;
+            const int b0 = dec_split_begin(g, chunk, j), b1 = dec_split_begin(g, chunk, j + 1);
+            items[atomicAdd(&s_off[bucket(b1 - b0)], 1)] =
+                make_int4(s, kvh | (j << 16), a.t_offset + b0 * kTile, j == g.n - 1 ? ctx : a.t_offset + b1 * kTile);
+        }
     }
 }
 
@@ -1003,6 +1037,8 @@ DecodePlan plan_decode(int32_t batch, int32_t num_kv_heads, int32_t max_context_
     p.chunk = (int32_t)chunk;
     p.max_splits = (int32_t)((max_context_len + chunk - 1) / chunk);
     if (p.max_splits < 1) p.max_splits = 1;
+    // the planning kernel cuts the last two chunks of a split pair into up to kTailPieces pieces
+    if (num_splits <= 0 && p.max_splits >= 2) p.max_splits += kTailPieces - 2;
     p.fixed = num_splits > 0;
     return p;
 }

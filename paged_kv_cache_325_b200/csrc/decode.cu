@@ -162,6 +162,25 @@ __device__ __forceinline__ int dec_split_begin(const SplitGeom &g, int chunk, in
     return g.nfull * chunk + k * g.base + min(k, g.extra);
 }
 
+// Output rows of (sequence s, KV head kvh) from its part_base partials alone (no tile of its own): the
+// element loop is strided over `nthreads` threads starting at `t0`.
+__device__ void plan_merge_bare(const DecodeArgs &a, int s, int kvh, int t0, int nthreads) {
+    const int G = a.group, D = a.head_dim;
+    for (int e = t0; e < G * D; e += nthreads) {
+        const int g = e / D, d = e % D, h = kvh * G + g;
+        const int64_t pb = ((int64_t)s * a.num_q_heads + h) * a.part_slots;
+        float m = -INFINITY;
+        for (int j = 0; j < a.part_base; ++j) m = fmaxf(m, __ldcg(a.part_lse + pb + j));
+        float num = 0.f, den = 0.f;
+        for (int j = 0; j < a.part_base; ++j) {
+            const float w = fast_exp2(__ldcg(a.part_lse + pb + j) - m);
+            num += w * __ldcg(a.part_o + (pb + j) * D + d);
+            den += w;
+        }
+        static_cast<__nv_bfloat16 *>(a.out)[(dec_row(a, s) * a.num_q_heads + h) * D + d] = __float2bfloat16_rn(num / den);
+    }
+}
+
 __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeArgs a, int32_t num_ctas) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");   // the decode kernel may start its set-up
     __shared__ unsigned long long s_total;
@@ -275,14 +294,25 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     // whole pairs: one thread each; split pairs go to a list (or, past its capacity, are written here)
     __shared__ int s_split[kPlanSplitList];
     __shared__ int s_nsplit;
-    if (tid == 0) s_nsplit = 0;
+    // pairs with no tiles after t_offset whose part_base partials the decode kernel would otherwise fold in
+    // (a shared-prefix sequence with no private token): merged here, a warp each
+    __shared__ int s_bare[kPlanSplitList];
+    __shared__ int s_nbare;
+    if (tid == 0) s_nsplit = s_nbare = 0;
     __syncthreads();
     for (int pr = tid; pr < npairs; pr += kPlanThreads) {
         const int s = pr / a.num_kv_heads, kvh = pr - s * a.num_kv_heads;
         const int tiles = s < kPlanCache ? s_tiles[s] : dec_tiles(a, s, false);
         const SplitGeom g = dec_split_geom(tiles, whole, chunk);
         if (a.merge_count) a.merge_count[pr] = g.n;   // splits of the pair still to finish (the decode counts down)
-        if (g.n == 0) continue;
+        if (g.n == 0) {
+            if (a.merge_count && a.part_base > 0 && tiles == 0 && dec_ctx(a, s) == a.t_offset && a.t_offset > 0) {
+                const int bi = atomicAdd(&s_nbare, 1);
+                if (bi < kPlanSplitList) s_bare[bi] = pr;
+                else plan_merge_bare(a, s, kvh, 0, 1);
+            }
+            continue;
+        }
         const int ctx = s < kPlanCache ? s_ctx[s] : dec_ctx(a, s);
         if (g.n == 1) {
             items[atomicAdd(&s_off[bucket(tiles)], 1)] = make_int4(s, kvh, a.t_offset, ctx);
@@ -325,6 +355,11 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
                 make_int4(s, kvh | (j << 16), a.t_offset + b0 * kTile, j == g.n - 1 ? ctx : a.t_offset + b1 * kTile);
         }
     }
+    const int nbare = min(s_nbare, kPlanSplitList);
+    for (int bi = tid >> 5; bi < nbare; bi += kPlanThreads / 32) {
+        const int pr = s_bare[bi];
+        plan_merge_bare(a, pr / a.num_kv_heads, pr % a.num_kv_heads, lane, 32);
+    }
 }
 
 struct DecItem {
@@ -335,6 +370,7 @@ struct DecItem {
 // used when the host plan cuts a pair into at most kMergeMaxSplits splits.
 constexpr int kMergeW = 1024;
 constexpr int kMergeMaxSplits = 8;
+constexpr int kFold = 8;             // earlier partials a pair's only item requests at once
 
 // A consumer-wide vote (the 128 threads of warps 0-3, named barrier 1): true iff v is true for all.
 __device__ __forceinline__ bool consumers_all(bool v) {
@@ -590,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         consumer_sync();
         const int4 pm = s_pend;
-        if (pm.z > 0) merge_pair<D>(a, pm.x, pm.y, pm.z, G, red_o, s_w, s_wsum);
+        if (pm.z > 0) merge_pair<D>(a, pm.x, pm.y, a.part_base + pm.z, G, red_o, s_w, s_wsum);
         consumer_sync();   // s_pend and the merge area are free again
     };
     for (;;) {
@@ -813,8 +849,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
         consumer_sync();
-        // the pair's only item and nothing merged in from elsewhere: write the result directly
-        const bool direct = a.part_base == 0 && it.t_begin == a.t_offset && it.t_end == it.ctx;
+        // the pair's only item: write the result directly -- merged with the part_base partials written before
+        // this launch (shared-prefix chunks) when there are some and this kernel merges
+        const bool only = it.t_begin == a.t_offset && it.t_end == it.ctx;
+        const bool direct = only && (a.part_base == 0 || a.merge_count);
         for (int e = threadIdx.x; e < G * D; e += kConsumerWarps * 32) {
             const int g = e / D, d = e % D;
             float mt = -INFINITY;
@@ -829,7 +867,38 @@ __global__ void __launch_bounds__(kThreads, 2)
                 ot += f * red_o[(w * G + g) * D + d];
             }
             const int h = it.kvh * G + g;
-            if (direct) {
+            if (direct && a.part_base > 0) {
+                // fold in the earlier partials of (s, h): log-sum-exp weights against this item's own.  The
+                // partials are requested kFold at a time, all before the first is used (one round trip each).
+                const int64_t pb = ((int64_t)it.s * a.num_q_heads + h) * a.part_slots;
+                const float lse_self = mt + __log2f(lt);
+                float m = lse_self, num = 0.f, den = 0.f, own = ot / lt;
+                for (int j0 = 0; j0 < a.part_base; j0 += kFold) {
+                    float pl[kFold], po[kFold];
+#pragma unroll
+                    for (int j = 0; j < kFold; ++j) {
+                        const bool in = j0 + j < a.part_base;
+                        pl[j] = in ? __ldcg(a.part_lse + pb + j0 + j) : -INFINITY;
+                        po[j] = in ? __ldcg(a.part_o + (pb + j0 + j) * D + d) : 0.f;
+                    }
+                    float mb = m;
+#pragma unroll
+                    for (int j = 0; j < kFold; ++j) mb = fmaxf(mb, pl[j]);
+                    const float c = fast_exp2(m - mb);   // rescale what was summed so far
+                    num *= c;
+                    den *= c;
+                    m = mb;
+#pragma unroll
+                    for (int j = 0; j < kFold; ++j) {
+                        const float w = fast_exp2(pl[j] - m);
+                        num += w * po[j];
+                        den += w;
+                    }
+                }
+                const float ws = fast_exp2(lse_self - m);
+                static_cast<__nv_bfloat16 *>(a.out)[(dec_row(a, it.s) * a.num_q_heads + h) * D + d] =
+                    __float2bfloat16_rn((num + ws * own) / (den + ws));
+            } else if (direct) {
                 static_cast<__nv_bfloat16 *>(a.out)[(dec_row(a, it.s) * a.num_q_heads + h) * D + d] =
                     __float2bfloat16_rn(ot / lt);
             } else {
@@ -1070,12 +1139,13 @@ DecodeWorkspace decode_workspace_layout(const DecodePlan &plan, int32_t batch, i
 cudaError_t launch_decode(const DecodeArgs &args, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                           cudaStream_t stream) {
     DecodeArgs a = args;
-    // Split pairs are merged in the split kernel when a pair has only a few splits and no partials come from
-    // elsewhere: that saves the combine launch, and each merge is short.  With many splits per pair (long
-    // contexts) the pairs' last splits finish together at the end of the grid, and a CTA per pair merging
-    // dozens of partials makes a longer tail than the combine kernel, which spreads the merge over many
-    // CTAs (measured: 4 splits per pair, -2 us; 32, +10 us).
-    a.merge_count = a.part_base == 0 && a.plan.max_splits > 1 && a.plan.max_splits <= kMergeMaxSplits
+    // Partials are merged in the split kernel when a pair has only a few splits: a pair's only item folds the
+    // part_base partials written before this launch (shared-prefix chunks) into its result, and the CTA that
+    // finishes a split pair's last split merges them all.  That saves the combine launch, and each merge is
+    // short.  With many splits per pair (long contexts) the pairs' last splits finish together at the end of
+    // the grid, and a CTA per pair merging dozens of partials makes a longer tail than the combine kernel,
+    // which spreads the merge over many CTAs (measured: 4 splits per pair, -2 us; 32, +10 us).
+    a.merge_count = (a.plan.max_splits > 1 || a.part_base > 0) && a.plan.max_splits <= kMergeMaxSplits
                         ? reinterpret_cast<int32_t *>(static_cast<char *>(a.plan_ws) +
                                                       decode_counter_offset(a.plan, a.batch, a.num_kv_heads))
                         : nullptr;

@@ -74,10 +74,10 @@ struct DecodeArgs {
     const int32_t *new_slots;
     void *k_cache, *v_cache;
     int64_t num_slots;
-    // set by launch_decode (callers leave it NULL): when no partials come from elsewhere (part_base == 0),
-    // the split kernel merges each split pair itself -- the CTA that finishes the pair's last split, counted
-    // in these per-pair counters (after the item table in plan_ws, zeroed by the planning kernel) -- and no
-    // combine kernel runs
+    // set by launch_decode (callers leave it NULL): when pairs have only a few splits, the split kernel merges
+    // the partials itself -- a pair's only item folds in the part_base partials, and the CTA that finishes a
+    // split pair's last split (counted down in these per-pair counters, after the item table in plan_ws, set
+    // by the planning kernel) merges all of them -- and no combine kernel runs
     int32_t *merge_count;
 };
 cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tm_k, const CUtensorMap &tm_v,

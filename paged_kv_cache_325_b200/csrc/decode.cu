@@ -92,6 +92,7 @@ struct DecPlanHdr {
     int32_t chunk;         // tiles per split of a longer pair
 };
 constexpr int kPlanHdrBytes = 256;
+constexpr int kDecSkip = -2;                // item.x of a first slot whose pair has no work (CTA takes the counter's)
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBuckets = 1024;          // item lengths (tiles) for the longest-first order; longer share the last
 constexpr int kPlanCache = 2048;            // sequences whose length the planning kernel keeps in shared memory
@@ -222,7 +223,10 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         chunk = (int)min((avg + 7) / 8, 1ull << 30);
         if (chunk < host_chunk) chunk = host_chunk;
     }
-    // longest-first order: count items per length bucket, then exclusive offsets from the longest bucket
+    // Item order: slots 0 .. n_first-1 hold the first split of pairs 0 .. n_first-1 (CTA c's first item, which
+    // its producer starts loading before this table exists), then every other item longest first: count those
+    // per length bucket, then exclusive offsets from the longest bucket
+    const int n_first = min(num_ctas, a.batch * a.num_kv_heads);
     auto bucket = [](int tiles) { return min(tiles, kPlanBuckets - 1); };
     for (int s = tid; s < a.batch; s += kPlanThreads) {
         const int tiles = s < kPlanCache ? s_tiles[s] : dec_tiles(a, s, false);
@@ -231,6 +235,8 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         if (g.nfull > 0) atomicAdd(&s_off[bucket(chunk)], g.nfull * a.num_kv_heads);
         if (g.extra > 0) atomicAdd(&s_off[bucket(g.base + 1)], g.extra * a.num_kv_heads);
         atomicAdd(&s_off[bucket(g.base)], (g.np - g.extra) * a.num_kv_heads);
+        const int nf = min(max(n_first - s * a.num_kv_heads, 0), a.num_kv_heads);   // first pairs of sequence s
+        if (nf > 0) atomicAdd(&s_off[bucket(dec_split_begin(g, chunk, 1))], -nf);
     }
     __syncthreads();
     {   // exclusive scan over the buckets from the longest down: thread t owns bucket kPlanBuckets - 1 - t
@@ -254,11 +260,11 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
             s_warp[lane] = t;               // inclusive totals of warps 0..lane
         }
         __syncthreads();
-        s_off[b] = inc - v + (w > 0 ? s_warp[w - 1] : 0);
+        s_off[b] = n_first + inc - v + (w > 0 ? s_warp[w - 1] : 0);
         if (tid == kPlanThreads - 1) {
             DecPlanHdr *h = reinterpret_cast<DecPlanHdr *>(a.plan_ws);
-            h->counter = num_ctas;          // item c < num_ctas is CTA c's first item (taken without the counter)
-            h->n_items = s_warp[kPlanThreads / 32 - 1];
+            h->counter = n_first;           // item c < n_first is CTA c's first item (taken without the counter)
+            h->n_items = n_first + s_warp[kPlanThreads / 32 - 1];
             h->whole = whole;
             h->chunk = chunk;
         }
@@ -311,11 +317,12 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
                 if (bi < kPlanSplitList) s_bare[bi] = pr;
                 else plan_merge_bare(a, s, kvh, 0, 1);
             }
+            if (pr < n_first) items[pr] = make_int4(kDecSkip, 0, 0, 0);   // CTA pr takes its first item from the counter
             continue;
         }
         const int ctx = s < kPlanCache ? s_ctx[s] : dec_ctx(a, s);
         if (g.n == 1) {
-            items[atomicAdd(&s_off[bucket(tiles)], 1)] = make_int4(s, kvh, a.t_offset, ctx);
+            items[pr < n_first ? pr : atomicAdd(&s_off[bucket(tiles)], 1)] = make_int4(s, kvh, a.t_offset, ctx);
             continue;
         }
         const int li = atomicAdd(&s_nsplit, 1);
@@ -326,7 +333,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         // past the list's capacity: this thread writes the pair's splits, one slot each
         for (int j = 0; j < g.n; ++j) {
             const int b0 = dec_split_begin(g, chunk, j), b1 = dec_split_begin(g, chunk, j + 1);
-            items[atomicAdd(&s_off[bucket(b1 - b0)], 1)] =
+            items[j == 0 && pr < n_first ? pr : atomicAdd(&s_off[bucket(b1 - b0)], 1)] =
                 make_int4(s, kvh | (j << 16), a.t_offset + b0 * kTile, j == g.n - 1 ? ctx : a.t_offset + b1 * kTile);
         }
     }
@@ -342,16 +349,19 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         const int ctx = s < kPlanCache ? s_ctx[s] : dec_ctx(a, s);
         const int ct = chunk * kTile;
         // the full chunks take consecutive slots of their bucket (lane 0 reserves them); each tail piece
-        // (lanes 0 .. np-1) reserves its own slot
+        // (lanes 0 .. np-1) reserves its own slot; split 0 of a first pair goes to its fixed slot
+        const bool first = pr < n_first;
+        const int j0 = first && g.nfull > 0 ? 1 : 0;   // full chunks from j0 on are bucketed
         int pos = 0;
-        if (lane == 0 && g.nfull > 0) pos = atomicAdd(&s_off[bucket(chunk)], g.nfull);
+        if (lane == 0 && g.nfull > j0) pos = atomicAdd(&s_off[bucket(chunk)], g.nfull - j0);
         pos = __shfl_sync(0xffffffffu, pos, 0);
-        for (int j = lane; j < g.nfull; j += 32)
-            items[pos + j] = make_int4(s, kvh | (j << 16), a.t_offset + j * ct, a.t_offset + (j + 1) * ct);
+        for (int j = j0 + lane; j < g.nfull; j += 32)
+            items[pos + j - j0] = make_int4(s, kvh | (j << 16), a.t_offset + j * ct, a.t_offset + (j + 1) * ct);
+        if (lane == 0 && j0 == 1) items[pr] = make_int4(s, kvh, a.t_offset, a.t_offset + ct);
         if (lane < g.np) {
             const int j = g.nfull + lane;
             const int b0 = dec_split_begin(g, chunk, j), b1 = dec_split_begin(g, chunk, j + 1);
-            items[atomicAdd(&s_off[bucket(b1 - b0)], 1)] =
+            items[j == 0 && first ? pr : atomicAdd(&s_off[bucket(b1 - b0)], 1)] =
                 make_int4(s, kvh | (j << 16), a.t_offset + b0 * kTile, j == g.n - 1 ? ctx : a.t_offset + b1 * kTile);
         }
     }
@@ -521,16 +531,66 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int B = a.block_size, box = a.box_tokens;
             uint32_t gt = 0, nqi = 0;             // tiles and Q copies issued so far
             bool ok = true;
+            const uint32_t qbytes = (uint32_t)(G * D * 2);
+            auto q_rows = [&](int s, int kvh) {   // Q rows of the GQA group: one contiguous bulk copy
+                return static_cast<const __nv_bfloat16 *>(a.q) + (dec_row(a, s) * a.num_q_heads + (int64_t)kvh * G) * D;
+            };
+            // the copies of one tile (tokens tile0 .. min(tile0 + kTile, t_end) - 1) into stage st
+            auto load_tile = [&](const int32_t *bt, int kvh, int tile0, int t_end, int st) {
+                const int nbox = (min(kTile, t_end - tile0) + box - 1) / box;
+                const uint32_t fb = smem_u32(full + st);
+                mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * 128 * C::kHalves * 2));
+                const uint32_t kdst = ring + st * C::kStageBytes;
+                const uint32_t vdst = kdst + C::kKvBytes;
+                for (int b = 0; b < nbox; ++b) {
+                    const int tok = tile0 + b * box;
+                    const int blk = __ldg(bt + tok / B);
+                    int row;
+                    if ((unsigned)blk < (unsigned)a.num_blocks) {
+                        row = blk * B + (tok % B);
+                    } else {               // out-of-range id: load zeros instead (TMA fills)
+                        report(a.dev_error, PA_DEVERR_BLOCK_ID);
+                        row = -box;
+                    }
+#pragma unroll
+                    for (int h = 0; h < C::kHalves; ++h) {
+                        const uint32_t off = h * kHalfBytes + b * box * 128;
+                        tma_load_3d(kdst + off, &tm_k, h * 64, kvh, row, fb);
+                        tma_load_3d(vdst + off, &tm_v, h * 64, kvh, row, fb);
+                    }
+                }
+            };
+            // CTA c < n_first owns the first split of pair c, which begins at t_offset whatever the plan cuts:
+            // its Q rows and first tile are requested before the planning kernel's table exists (they are
+            // inputs the planning kernel does not write: a fused store's new token lies past the first tile)
+            const int n_first = min((int)gridDim.x, a.batch * a.num_kv_heads);
+            bool pre = false;
+            if ((int)blockIdx.x < n_first) {
+                const int s0 = blockIdx.x / a.num_kv_heads, kvh0 = blockIdx.x % a.num_kv_heads;
+                if (dec_tiles(a, s0, false) > 0 && dec_ctx(a, s0) - a.t_offset > kTile) {
+                    pre = true;
+                    mbar_expect_tx(smem_u32(qfull), qbytes);   // the arrival comes with the item, after the table
+                    bulk_load(qsm, q_rows(s0, kvh0), qbytes, smem_u32(qfull));
+                    load_tile(a.block_table + (int64_t)s0 * a.bt_stride, kvh0, a.t_offset, dec_ctx(a, s0), 0);
+                    gt = 1;
+                }
+            }
             asm volatile("griddepcontrol.wait;" ::: "memory");   // the planning kernel's table is complete
             DecPlanHdr *hdr = reinterpret_cast<DecPlanHdr *>(a.plan_ws);
             const int4 *items = reinterpret_cast<const int4 *>(reinterpret_cast<const char *>(a.plan_ws) + kPlanHdrBytes);
             const int n_items = __ldcg(&hdr->n_items);
             const int4 kEnd = make_int4(-1, 0, 0, 0);
-            int idx = blockIdx.x;               // the first item is this CTA's own; the rest come from the counter
+            // the first item is this CTA's own slot (if it has one); the rest come from the counter
+            int idx = (int)blockIdx.x < n_first ? (int)blockIdx.x : atomicAdd(&hdr->counter, 1);
             int4 d = idx < n_items ? __ldcg(items + idx) : kEnd;
             while (ok) {
                 const int qs = nqi & 1;
                 if (nqi >= 2 && !mbar_wait(smem_u32(qempty + qs), ((nqi >> 1) - 1) & 1, a.dev_error)) break;
+                if (d.x == kDecSkip) {            // a first slot whose pair has no work
+                    idx = atomicAdd(&hdr->counter, 1);
+                    d = idx < n_items ? __ldcg(items + idx) : kEnd;
+                    continue;
+                }
                 if (d.x < 0) {                    // end of the stream: an item with s < 0, no copy
                     desc[qs] = d;
                     mbar_arrive(smem_u32(qfull + qs));
@@ -542,47 +602,35 @@ __global__ void __launch_bounds__(kThreads, 2)
                 desc[qs] = d;                     // the item rides in the Q slot's descriptor
                 const int s = d.x, kvh = d.y & 0xffff, t_begin = d.z, t_end = d.w;
                 const int ntiles = (t_end - t_begin + kTile - 1) / kTile;
-                // Q rows of the GQA group: one contiguous bulk copy
-                const uint32_t qbytes = (uint32_t)(G * D * 2);
-                mbar_arrive_expect_tx(smem_u32(qfull + qs), qbytes);
-                bulk_load(qsm + qs * qslot,
-                          static_cast<const __nv_bfloat16 *>(a.q) + (dec_row(a, s) * a.num_q_heads + (int64_t)kvh * G) * D,
-                          qbytes, smem_u32(qfull + qs));
+                int t_start = 0;
+                if (pre) {
+                    // this is pair blockIdx.x's first split (its slot), whose Q rows and first tile are on their
+                    // way: the arrival completes the Q slot with the item written
+                    pre = false;
+                    mbar_arrive(smem_u32(qfull + qs));
+                    t_start = 1;
+                } else {
+                    mbar_arrive_expect_tx(smem_u32(qfull + qs), qbytes);
+                    bulk_load(qsm + qs * qslot, q_rows(s, kvh), qbytes, smem_u32(qfull + qs));
+                }
                 ++nqi;
                 const int32_t *bt = a.block_table + (int64_t)s * a.bt_stride;
-                for (int t = 0; t < ntiles; ++t, ++gt) {
+                for (int t = t_start; t < ntiles; ++t, ++gt) {
                     const int st = gt % C::kStages;
                     if (gt >= (uint32_t)C::kStages &&
                         !mbar_wait(smem_u32(empty + st), ((gt / C::kStages) & 1) ^ 1, a.dev_error)) {
                         ok = false;
                         break;
                     }
-                    const int tile0 = t_begin + t * kTile;
-                    const int nbox = (min(kTile, t_end - tile0) + box - 1) / box;
-                    const uint32_t fb = smem_u32(full + st);
-                    mbar_arrive_expect_tx(fb, (uint32_t)(nbox * box * 128 * C::kHalves * 2));
-                    const uint32_t kdst = ring + st * C::kStageBytes;
-                    const uint32_t vdst = kdst + C::kKvBytes;
-                    for (int b = 0; b < nbox; ++b) {
-                        const int tok = tile0 + b * box;
-                        const int blk = __ldg(bt + tok / B);
-                        int row;
-                        if ((unsigned)blk < (unsigned)a.num_blocks) {
-                            row = blk * B + (tok % B);
-                        } else {               // out-of-range id: load zeros instead (TMA fills)
-                            report(a.dev_error, PA_DEVERR_BLOCK_ID);
-                            row = -box;
-                        }
-#pragma unroll
-                        for (int h = 0; h < C::kHalves; ++h) {
-                            const uint32_t off = h * kHalfBytes + b * box * 128;
-                            tma_load_3d(kdst + off, &tm_k, h * 64, kvh, row, fb);
-                            tma_load_3d(vdst + off, &tm_v, h * 64, kvh, row, fb);
-                        }
-                    }
+                    load_tile(bt, kvh, t_begin + t * kTile, t_end, st);
                     // the next item: index and record, issued now and used when this item's copies are out
-                    if (t == max(0, ntiles - 3)) idx_next = atomicAdd(&hdr->counter, 1);
-                    if (t == max(0, ntiles - 2)) d_next = idx_next < n_items ? __ldcg(items + idx_next) : kEnd;
+                    if (t == max(t_start, ntiles - 3)) idx_next = atomicAdd(&hdr->counter, 1);
+                    if (t == max(t_start, ntiles - 2)) d_next = idx_next < n_items ? __ldcg(items + idx_next) : kEnd;
+                }
+                // an item whose every tile was loaded before the table (one tile) still takes the next item
+                if (t_start >= ntiles) {
+                    idx_next = atomicAdd(&hdr->counter, 1);
+                    d_next = idx_next < n_items ? __ldcg(items + idx_next) : kEnd;
                 }
                 d = d_next;
             }

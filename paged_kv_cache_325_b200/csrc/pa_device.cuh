@@ -51,6 +51,11 @@ PA_DEVICE void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
                  : "memory");
 }
 
+// Post expected bytes without arriving (the arrival comes later, from the same or another thread).
+PA_DEVICE void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
 PA_DEVICE bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(

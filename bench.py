@@ -230,6 +230,33 @@ def capture(fn):
     return g.replay, g
 
 
+def count_kernels(fn):
+    """Kernel launches one call of fn makes: fn is captured on a side stream with the runtime API (nothing runs)
+    and the kernel nodes of the captured graph are counted."""
+    from cuda.bindings import runtime as rt
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        (err,) = rt.cudaStreamBeginCapture(s.cuda_stream, rt.cudaStreamCaptureMode.cudaStreamCaptureModeRelaxed)
+        assert err == rt.cudaError_t.cudaSuccess, err
+        try:
+            fn()
+        finally:
+            err, graph = rt.cudaStreamEndCapture(s.cuda_stream)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    try:
+        err, _, n = rt.cudaGraphGetNodes(graph, 0)
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+        assert err == rt.cudaError_t.cudaSuccess, err
+        kernels = 0
+        for node in nodes[:n]:
+            err, ty = rt.cudaGraphNodeGetType(node)
+            kernels += int(ty == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+        return kernels
+    finally:
+        rt.cudaGraphDestroy(graph)
+
+
 class DecodeBench:
     def __init__(self, case, device):
         import paged_kv_cache_325_b200 as pa
@@ -317,7 +344,9 @@ def bench_primary(args, world, rank, device, pk):
         "roofline": {"kernel": "decode_split_kernel<128> (store fused)", "bound": "hbm",
                      "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                      "traffic": recorded_traffic("store_decode_qwen3_0.6b"), "alg_bytes_per_launch": alg},
-        "gpu_launches": 3 * args.steps,     # per step: planning, decode (store fused in) and combine kernels
+        # per step: the kernels of one pa_store_kv_decode call (planning, decode with the store fused in, and a
+        # combine only when pairs have many splits), counted from a captured graph of the call
+        "gpu_launches": count_kernels(b.store_decode) * args.steps,
         "clocks": clocks,
     }
     # the same step as two launches (pa_store_kv, then pa_decode), for comparison; rank 0 at N=1

@@ -33,6 +33,20 @@ def test_decode_workloads_full_size(cuda_lib, make):
     assert_close(out, ref, what=case.name)
 
 
+@pytest.mark.parametrize("ctx,what", [
+    # one long context among short ones: the long pairs are cut into chunks plus four smaller tail pieces
+    # (7 splits: merged inside the decode kernel by the CTA that finishes the last one) ...
+    ([1200] + [64] * 60, "merged in the decode kernel"),
+    # ... and with many splits per pair (14: merged by the combine kernel); fewer (sequence, KV head) pairs
+    # than CTAs, so most CTAs start on the counter instead of a pair of their own
+    ([6000] + [64] * 100, "merged by the combine kernel"),
+])
+def test_decode_skewed_batch_auto_splits(cuda_lib, ctx, what):
+    case = W.make_decode_case(ctx, 8, 2, 128, 64, seed=310 + len(ctx))
+    _, out = _run(case)
+    assert_close(out, oracle_decode(case), what=what)
+
+
 @pytest.mark.parametrize("num_splits", [1, 2, 3, 5, 16])
 def test_decode_explicit_splits(cuda_lib, num_splits):
     case = W.make_decode_case([1, 63, 64, 65, 200, 511, 777, 1024], 8, 2, 128, 64, seed=300 + num_splits)

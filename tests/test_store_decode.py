@@ -47,6 +47,19 @@ def test_store_decode_workloads(cuda_lib, make):
     _cache_equals_oracle_store(g, case)
 
 
+@pytest.mark.parametrize("ctx", [[1200] + [64] * 60, [6000] + [64] * 100], ids=["few_splits", "many_splits"])
+def test_store_decode_skewed_batch_auto_splits(cuda_lib, ctx):
+    """Store fused into a decode whose plan splits the long pair (merged in the kernel, or by the combine):
+    the long sequence's CTA starts on its first tile before the plan exists, the short ones (one tile,
+    which holds their new token) do not."""
+    case = W.make_decode_case(ctx, 8, 2, 128, 64, seed=1610 + len(ctx))
+    g = DecodeOnGpu(case)
+    out = _fused(g)
+    torch.cuda.synchronize()
+    assert_close(out, oracle_decode(case), what=f"{len(ctx)} sequences")
+    _cache_equals_oracle_store(g, case)
+
+
 @pytest.mark.parametrize("B", [16, 32, 64, 128, 256])
 @pytest.mark.parametrize("Hq,Hkv,D", [(8, 4, 128), (32, 8, 64), (6, 1, 64), (16, 16, 128)])
 def test_store_decode_shapes(cuda_lib, B, Hq, Hkv, D):

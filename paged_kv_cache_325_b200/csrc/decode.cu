@@ -561,20 +561,32 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
             };
             // CTA c < n_first owns the first split of pair c, which begins at t_offset whatever the plan cuts:
-            // its Q rows and first tile are requested before the planning kernel's table exists (they are
-            // inputs the planning kernel does not write: a fused store's new token lies past the first tile)
+            // its Q rows and first tiles are requested before the planning kernel's table exists.  They are
+            // inputs the planning kernel does not write (a fused store's new token lies past them), and never
+            // more tiles than any first split of the pair can have: all of a pair of at most 4 tiles (never
+            // split: the plan keeps pairs up to the per-CTA average, at least 4 tiles, whole), 2 of a longer
+            // one (a first chunk has at least 4, a first tail piece at least 2), the chunk when the caller
+            // fixed the split count; at most one ring's worth.
             const int n_first = min((int)gridDim.x, a.batch * a.num_kv_heads);
-            bool pre = false;
+            int npre = 0;
             if ((int)blockIdx.x < n_first) {
                 const int s0 = blockIdx.x / a.num_kv_heads, kvh0 = blockIdx.x % a.num_kv_heads;
-                if (dec_tiles(a, s0, false) > 0 && dec_ctx(a, s0) - a.t_offset > kTile) {
-                    pre = true;
+                const int tiles0 = dec_tiles(a, s0, false);
+                if (tiles0 > 0) {
+                    const int ctx0 = dec_ctx(a, s0);
+                    const int before_new = (ctx0 - 1 - a.t_offset) / kTile;   // tiles before the new token's
+                    const int split_min = a.plan.fixed ? a.plan.chunk / kTile : (tiles0 <= 4 ? tiles0 : 2);
+                    npre = min(min(C::kStages, before_new), split_min);
+                }
+                if (npre > 0) {
                     mbar_expect_tx(smem_u32(qfull), qbytes);   // the arrival comes with the item, after the table
                     bulk_load(qsm, q_rows(s0, kvh0), qbytes, smem_u32(qfull));
-                    load_tile(a.block_table + (int64_t)s0 * a.bt_stride, kvh0, a.t_offset, dec_ctx(a, s0), 0);
-                    gt = 1;
+                    for (int t = 0; t < npre; ++t)
+                        load_tile(a.block_table + (int64_t)s0 * a.bt_stride, kvh0, a.t_offset + t * kTile, dec_ctx(a, s0), t);
+                    gt = (uint32_t)npre;
                 }
             }
+            bool pre = npre > 0;
             asm volatile("griddepcontrol.wait;" ::: "memory");   // the planning kernel's table is complete
             DecPlanHdr *hdr = reinterpret_cast<DecPlanHdr *>(a.plan_ws);
             const int4 *items = reinterpret_cast<const int4 *>(reinterpret_cast<const char *>(a.plan_ws) + kPlanHdrBytes);
@@ -604,11 +616,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int ntiles = (t_end - t_begin + kTile - 1) / kTile;
                 int t_start = 0;
                 if (pre) {
-                    // this is pair blockIdx.x's first split (its slot), whose Q rows and first tile are on their
+                    // this is pair blockIdx.x's first split (its slot), whose Q rows and first tiles are on their
                     // way: the arrival completes the Q slot with the item written
                     pre = false;
                     mbar_arrive(smem_u32(qfull + qs));
-                    t_start = 1;
+                    t_start = npre;
                 } else {
                     mbar_arrive_expect_tx(smem_u32(qfull + qs), qbytes);
                     bulk_load(qsm + qs * qslot, q_rows(s, kvh), qbytes, smem_u32(qfull + qs));

@@ -664,9 +664,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(smem_u32(s_full + x), ns & 1, a.dev_error, 0xffffffffu, abort_flag)) { ok = false; break; }
                 ++ns;
                 tc_fence_after();
-                uint32_t sr[4][32];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) tmem_ld32(lane_base + col_s(x) + q * 32, sr[q]);
+                uint32_t sr[4][32];   // the S row: one 128-column TMEM load (measured ~2 % faster than four)
+                tmem_ld128(lane_base + col_s(x), reinterpret_cast<uint32_t (&)[128]>(sr));
                 tc_wait_ld();
                 const int thr = lim - (U.kbeg + j * kN);   // keys e <= thr are visible
                 // row maximum: three-input max over pairs, four independent chains
@@ -695,16 +694,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     rescale = true;
                 }
                 // P = exp2(s * scale_log2 - m_ref) as packed bf16 pairs, written over the S_X columns already
-                // read (32 keys = 16 columns per store); the scaling runs on pairs (f32x2 FMA).  The row sum
+                // read (64 keys = 32 columns per store); the scaling runs on pairs (f32x2 FMA).  The row sum
                 // adds the bf16 values the PV product multiplies, not the fp32 ones, so that the weights of the
                 // numerator and the denominator are the same numbers: with the lazy maximum the largest P is not
                 // a power of two, and its rounding would otherwise show in the output of a row that one key
                 // dominates.
                 const uint64_t sl2 = f2_pack(sl, sl), neg2 = f2_pack(-m_ref, -m_ref);
                 uint64_t ls2[2] = {0ull, 0ull};
+                uint32_t w2[32];   // P of 64 keys (32 columns), stored with one instruction per pair of chunks
 #pragma unroll
                 for (int kc = 0; kc < kN / 32; ++kc) {
-                    uint32_t w[16];
+                    uint32_t *w = w2 + (kc & 1) * 16;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const uint64_t x2 =
@@ -721,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ls2[i & 1] = f2_add(ls2[i & 1], f2_pack(__uint_as_float(w[i] << 16),
                                                                 __uint_as_float(w[i] & 0xffff0000u)));
                     }
-                    tmem_st16(lane_base + col_s(x) + kc * 16, w);
+                    if (kc & 1) tmem_st32(lane_base + col_s(x) + (kc - 1) * 16, w2);
                 }
                 float ls[4];
                 f2_unpack(ls2[0], ls[0], ls[1]);

@@ -115,8 +115,9 @@ PA_API pa_status pa_store_kv(const void *k, const void *v, int64_t k_row_stride,
 
 /*
  * Bytes of device workspace pa_decode needs for these sizes on the current
- * device (0 only when batch <= 0): the planning kernel's table of work items
- * and, when a context may be split, the per-split partial results.
+ * device (0 only when batch <= 0): the planning kernel's table of work items,
+ * a counter per (sequence, KV head) and, when a context may be split, the
+ * per-split partial results.
  */
 PA_API size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                 int32_t max_context_len, int32_t block_size);
@@ -145,11 +146,15 @@ PA_API size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32
  *                    initialisation and are garbage afterwards.  Two calls
  *                    whose kernels may overlap on the GPU need two workspaces.
  *
- * Three kernels on `stream`: a one-CTA planning kernel reads context_lens and
- * writes a longest-first table of work items (a whole (sequence, KV head), or
- * one split of a context far longer than the average per-CTA load); the
- * persistent decode kernel takes items from it with an atomic counter; a
- * combine kernel merges the partial results of split contexts by log-sum-exp.
+ * Two or three kernels on `stream`: a one-CTA planning kernel reads
+ * context_lens and writes a table of work items (a whole (sequence, KV head),
+ * or one split of a context far longer than the average per-CTA load): the
+ * first split of pair c for decode CTA c, which starts on it before the table
+ * exists, then the rest longest first; the persistent decode kernel takes
+ * items with an atomic counter.  Partial results of split contexts are merged
+ * by log-sum-exp: inside the decode kernel, by the CTA that finishes a pair's
+ * last split, when the plan allows at most 8 splits per pair; otherwise by a
+ * third, combine kernel.
  */
 PA_API pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
                     const int32_t *block_table, int32_t block_table_stride, const int32_t *context_lens,
@@ -224,7 +229,10 @@ PA_API pa_status pa_decode_split(void *out, const void *q, const void *k_cache, 
  *      each chunk giving an fp32 partial and its log-sum-exp;
  *   2. the split-KV decode covers each sequence's private tokens
  *      [num_shared_blocks * block_size, context_lens[s]);
- *   3. all partials of a (sequence, q-head) are merged by log-sum-exp.
+ *   3. all partials of a (sequence, q-head) are merged by log-sum-exp (in the
+ *      decode kernel when its plan gives at most 8 splits per pair, else by a
+ *      combine kernel; a sequence with no private token by the planning
+ *      kernel).
  * Every context_lens[s] must be >= num_shared_blocks * block_size (checked
  * mode reports PA_DEVERR_CONTEXT_LEN; a table row whose first blocks differ
  * from row 0's is reported as PA_DEVERR_BLOCK_ID).  The GQA group must divide

@@ -209,8 +209,9 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
     if ((tid & 31) == 0) atomicAdd(&s_total, part);
     __syncthreads();
-    // split rule: pairs up to the average per-CTA load stay whole; longer ones are cut into pieces of an
-    // eighth of it (never finer than the host's chunk, which sized the partial slots)
+    // split rule: pairs up to the average per-CTA load stay whole; longer ones are cut into pieces of a
+    // quarter of it (never finer than the host's chunk, which sized the partial slots; an eighth measured 2 us
+    // slower at long context: more partials to merge, and the tail pieces already even out the ends)
     int whole, chunk;
     const int host_chunk = a.plan.chunk / kTile;
     if (a.plan.fixed) {
@@ -220,7 +221,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         const unsigned long long avg = (s_total + num_ctas - 1) / (unsigned long long)num_ctas;
         whole = (int)min(avg, 1ull << 30);
         if (whole < 4) whole = 4;
-        chunk = (int)min((avg + 7) / 8, 1ull << 30);
+        chunk = (int)min((avg + 3) / 4, 1ull << 30);
         if (chunk < host_chunk) chunk = host_chunk;
     }
     // Item order: slots 0 .. n_first-1 hold the first split of pairs 0 .. n_first-1 (CTA c's first item, which

@@ -64,8 +64,8 @@ struct PrefillCfg {
     static constexpr int kStageBytes = kFused ? kStageTokens * 4 * D : 0;
     static constexpr int kBarOff = kStageOff + kStageBytes;
     // kv_full[S] kv_empty[S] q_full q_empty s_full[2] p_full[2] o_full[2] o_empty[2] done uq_full[4] uq_empty[4]
-    // v_fixed[kFixRing] vlast_full[kVlast] vlast_empty[kVlast] cp_full
-    static constexpr int kNumBars = 2 * kSlots + 11 + 2 * kUnitQueue + kFixRing + 2 * kVlast + 1;
+    // v_fixed[kFixRing] vlast_full[kVlast] vlast_empty[kVlast] cp_full epi_done[2]
+    static constexpr int kNumBars = 2 * kSlots + 11 + 2 * kUnitQueue + kFixRing + 2 * kVlast + 1 + 2;
     static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 64 + kUnitQueue * 64 + 1024;
     static constexpr uint32_t kTmemCols = 512;                  // S_A 0, O_A 128, S_B 256, O_B 384
                                                                 // (P_X, bf16, overwrites the first 64 columns of S_X)
@@ -127,7 +127,9 @@ __device__ __forceinline__ Unit unit_from_record(const PrefillArgs &a, int4 rec,
 
 // kFused: pa_store_kv_prefill_varlen.  Keys past the cached prefix come from the new K/V rows (tm_kn, tm_vn)
 // instead of the cache, and the V-fix warp stores each unit's own new rows to their cache slots.
-template <int D, bool kFused>
+// kPartial: the key range is cut into chunks and each writes fp32 partials with their log-sum-exp (a.part_o,
+// a.part_lse) instead of bf16 rows (the shared-prefix phase of pa_decode_shared_prefix).
+template <int D, bool kFused, bool kPartial>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kn,
@@ -154,6 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *vlast_full = v_fixed + kFixRing;    // [kVlast]
     uint64_t *vlast_empty = vlast_full + kVlast;  // [kVlast]
     uint64_t *cp_full = vlast_empty + kVlast;     // fused store: a copy round's rows are in the staging area
+    // partial results: softmax warpgroup X has written its tile's partials out of the Q_X buffer (the next unit's
+    // Q may be loaded over it)
+    uint64_t *epi_done = cp_full + 1;             // [2]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
     // set by the first wait of this CTA that gives up; every other wait then gives up at once
     volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(tmem_slot + 1);
@@ -191,6 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(vlast_empty + i), 1);
         }
         mbar_init(smem_u32(cp_full), 1);
+        for (int x = 0; x < 2; ++x) mbar_init(smem_u32(epi_done + x), 4);
         for (int i = 0; i < kUnitQueue; ++i) {
             mbar_init(smem_u32(uq_full + i), 1);
             mbar_init(smem_u32(uq_empty + i), 11);  // the MMA, V-fix and Q warps, the eight softmax warps
@@ -353,13 +359,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (warp == kQWarp) {
             // ============================================================== Q ==
             // Both Q tiles of each unit, as soon as the previous unit's S products have read the buffer.
+            // With partial results (kPartial) the softmax warpgroups stage their epilogue in the Q buffer, so a
+            // unit's Q also waits until the previous unit's tiles have been written out of it.
             if (lane == 0) tma_prefetch_desc(&tm_q);
-            uint32_t nq = 0;
+            uint32_t nq = 0, ne[2] = {0, 0};
+            int prev_nt[2] = {0, 0};
             for (uint32_t k = 0;; ++k) {
                 Unit U;
                 if (!pop_unit(k, lane == 0, U)) break;
                 if (!U.valid) continue;
                 if (nq > 0 && !mbar_wait(smem_u32(q_empty), (nq - 1) & 1, a.dev_error, 0xffffffffu, abort_flag)) break;
+                bool epi_ok = true;
+                for (int x = 0; x < 2 && epi_ok; ++x)
+                    if (kPartial && prev_nt[x] > 0) {
+                        epi_ok = mbar_wait(smem_u32(epi_done + x), ne[x] & 1, a.dev_error, 0xffffffffu, abort_flag);
+                        ++ne[x];
+                    }
+                if (!epi_ok) break;
+                prev_nt[0] = U.nt[0];
+                prev_nt[1] = U.nt[1];
                 if (lane == 0) {
                     mbar_arrive_expect_tx(smem_u32(q_full), (uint32_t)(2 * C::kTileBytes));
                     for (int x = 0; x < 2; ++x)
@@ -757,40 +775,76 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) +
                                                    ((int64_t)(U.q0 + (store ? t : 0)) * a.num_q_heads +
                                                     (int64_t)U.kvh * G + r % G) * D);
-            uint32_t o[D / 32][32];
-#pragma unroll
-            for (int q = 0; q < D / 32; ++q) tmem_ld32(lane_base + col_o(x) + q * 32, o[q]);
-            tc_wait_ld();
-            // O_X is in registers: hand its TMEM columns back to the MMA thread now, so that the next unit's
-            // first PV product does not wait for the global stores below
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(o_empty + x));
-            if (store && a.part_o) {
+            if (kPartial) {
                 // partial result of this key chunk: fp32 O / l and its log-sum-exp (log2 units), to be merged
-                // with the other partials of the same (query, head)
-                const int64_t pi = ((int64_t)(U.q0 + t) * a.num_q_heads + (int64_t)U.kvh * G + r % G) * a.part_slots +
-                                   a.part_base + U.chunk;
-                float4 *po = reinterpret_cast<float4 *>(a.part_o + pi * D);
+                // with the other partials of the same (query, head).  A thread holds one 512-byte row; written
+                // straight out, every warp store would touch 32 rows.  So the warp stages 32 columns of its 32
+                // rows at a time in its 4 KB of the Q_X buffer (free: every S product of this unit has completed
+                // before o_full; the Q warp waits for epi_done before loading over it), 16-byte pieces swizzled
+                // by row so that neither side conflicts on banks, and reads them back four rows per instruction:
+                // each store instruction then writes four whole 128-byte lines.
+                const int64_t pi = store ? ((int64_t)(U.q0 + t) * a.num_q_heads + (int64_t)U.kvh * G + r % G) *
+                                               a.part_slots + a.part_base + U.chunk
+                                         : 0;
+                const uint32_t smask = __ballot_sync(0xffffffffu, store);
+                const uint32_t stg = q_s + (uint32_t)(x * C::kTileBytes) + (uint32_t)((warp & 3) * 4096);
+                const int c = lane & 7;
+#pragma unroll 1
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t oq[32];   // 32 columns of O_X at a time (units per CTA are few here: O_X is released after)
+                    tmem_ld32(lane_base + col_o(x) + q * 32, oq);
+                    tc_wait_ld();
 #pragma unroll
-                for (int q = 0; q < D / 32; ++q)
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        po[(q * 32 + e) / 4] = make_float4(__uint_as_float(o[q][e]) * inv, __uint_as_float(o[q][e + 1]) * inv,
-                                                           __uint_as_float(o[q][e + 2]) * inv, __uint_as_float(o[q][e + 3]) * inv);
-                a.part_lse[pi] = m_ref + __log2f(l);
-            } else if (store) {
-#pragma unroll
-                for (int q = 0; q < D / 32; ++q)
-#pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        uint4 v;
-                        v.x = pack_bf16(__uint_as_float(o[q][e]) * inv, __uint_as_float(o[q][e + 1]) * inv);
-                        v.y = pack_bf16(__uint_as_float(o[q][e + 2]) * inv, __uint_as_float(o[q][e + 3]) * inv);
-                        v.z = pack_bf16(__uint_as_float(o[q][e + 4]) * inv, __uint_as_float(o[q][e + 5]) * inv);
-                        v.w = pack_bf16(__uint_as_float(o[q][e + 6]) * inv, __uint_as_float(o[q][e + 7]) * inv);
-                        dst[(q * 32 + e) / 8] = v;
+                    for (int e = 0; e < 8; ++e)
+                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(stg + lane * 128 + ((e ^ (lane & 7)) << 4)),
+                                     "f"(__uint_as_float(oq[4 * e]) * inv), "f"(__uint_as_float(oq[4 * e + 1]) * inv),
+                                     "f"(__uint_as_float(oq[4 * e + 2]) * inv), "f"(__uint_as_float(oq[4 * e + 3]) * inv)
+                                     : "memory");
+                    __syncwarp();
+#pragma unroll 4
+                    for (int i = 0; i < 8; ++i) {
+                        const int rr = i * 4 + (lane >> 3);          // the warp's row this lane writes 16 bytes of
+                        const int64_t pr = __shfl_sync(0xffffffffu, pi, rr);
+                        float4 v;
+                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                                     : "r"(stg + rr * 128 + ((c ^ (rr & 7)) << 4))
+                                     : "memory");
+                        if ((smask >> rr) & 1) reinterpret_cast<float4 *>(a.part_o + pr * D + q * 32)[c] = v;
                     }
+                    __syncwarp();
+                }
+                tc_fence_before();
+                if (store) a.part_lse[pi] = m_ref + __log2f(l);
+                fence_proxy_async_smem();   // the next Q copy (async proxy) lands where this warp wrote
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(o_empty + x));
+                    mbar_arrive(smem_u32(epi_done + x));
+                }
+            } else {
+                uint32_t o[D / 32][32];
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q) tmem_ld32(lane_base + col_o(x) + q * 32, o[q]);
+                tc_wait_ld();
+                // O_X is in registers: hand its TMEM columns back to the MMA thread now, so that the next unit's
+                // first PV product does not wait for the global stores below
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(o_empty + x));
+                if (store) {
+#pragma unroll
+                    for (int q = 0; q < D / 32; ++q)
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            uint4 v;
+                            v.x = pack_bf16(__uint_as_float(o[q][e]) * inv, __uint_as_float(o[q][e + 1]) * inv);
+                            v.y = pack_bf16(__uint_as_float(o[q][e + 2]) * inv, __uint_as_float(o[q][e + 3]) * inv);
+                            v.z = pack_bf16(__uint_as_float(o[q][e + 4]) * inv, __uint_as_float(o[q][e + 5]) * inv);
+                            v.w = pack_bf16(__uint_as_float(o[q][e + 6]) * inv, __uint_as_float(o[q][e + 7]) * inv);
+                            dst[(q * 32 + e) / 8] = v;
+                        }
+                }
             }
         }
     }
@@ -809,14 +863,16 @@ cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &tm_q, cons
                              const CUtensorMap &tm_v, const CUtensorMap &tm_kn, const CUtensorMap &tm_vn,
                              cudaStream_t stream) {
     const bool fused = a.new_slots != nullptr;
-    auto kernel = fused ? prefill_kernel<D, true> : prefill_kernel<D, false>;
+    const int mode = fused ? 1 : a.part_o ? 2 : 0;
+    auto kernel = mode == 1 ? prefill_kernel<D, true, false> : mode == 2 ? prefill_kernel<D, false, true>
+                                                                          : prefill_kernel<D, false, false>;
     const int smem_bytes = fused ? PrefillCfg<D, true>::kSmemBytes : PrefillCfg<D, false>::kSmemBytes;
-    static std::atomic<uint64_t> configured[2] = {{0}, {0}};
+    static std::atomic<uint64_t> configured[3] = {{0}, {0}, {0}};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const uint64_t bit = uint64_t(1) << (dev & 63);
-    if (!(configured[fused].load(std::memory_order_acquire) & bit)) {
+    if (!(configured[mode].load(std::memory_order_acquire) & bit)) {
         // the register split inside the kernel assumes the launch-time count it was written for
         cudaFuncAttributes fa;
         e = cudaFuncGetAttributes(&fa, kernel);
@@ -824,7 +880,7 @@ cudaError_t launch_prefill_d(const PrefillArgs &a, const CUtensorMap &tm_q, cons
         if ((uint32_t)fa.numRegs * kThreads < 2 * 128 * kRegsSoftmax + 128 * kRegsOther) return cudaErrorNotSupported;
         e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
         if (e != cudaSuccess) return e;
-        configured[fused].fetch_or(bit, std::memory_order_acq_rel);
+        configured[mode].fetch_or(bit, std::memory_order_acq_rel);
     }
     const int TQ = kM / a.group;
     const size_t plan_smem = (size_t)2 * a.batch * sizeof(int32_t);

@@ -94,7 +94,8 @@ struct DecPlanHdr {
 constexpr int kPlanHdrBytes = 256;
 constexpr int kDecSkip = -2;                // item.x of a first slot whose pair has no work (CTA takes the counter's)
 constexpr int kPlanThreads = 1024;
-constexpr int kPlanBuckets = 1024;          // item lengths (tiles) for the longest-first order; longer share the last
+constexpr int kPlanBuckets = 1024;
+constexpr int kDecLocalCut = 1024;          // batches up to this many sequences: each CTA cuts its first item itself          // item lengths (tiles) for the longest-first order; longer share the last
 constexpr int kPlanCache = 2048;            // sequences whose length the planning kernel keeps in shared memory
 constexpr int kPlanSplitList = 1024;        // split (sequence, KV head) pairs whose items a warp each writes
 
@@ -163,6 +164,35 @@ __device__ __forceinline__ int dec_split_begin(const SplitGeom &g, int chunk, in
     return g.nfull * chunk + k * g.base + min(k, g.extra);
 }
 
+// The split rule, from the total work in tiles over the grid's CTAs: pairs up to the average per-CTA load stay
+// whole; longer ones are cut into pieces of a quarter of it (never finer than the host's chunk, which sized the
+// partial slots; an eighth measured 2 us slower at long context: more partials to merge, and the tail pieces
+// already even out the ends).  The planning kernel and each decode CTA (for its first item) apply it to the
+// same total, so they cut every pair the same way.
+__device__ __forceinline__ void dec_cut(const DecodeArgs &a, unsigned long long total, int num_ctas, int &whole,
+                                        int &chunk) {
+    const int host_chunk = a.plan.chunk / kTile;
+    if (a.plan.fixed) {
+        whole = 0;
+        chunk = host_chunk;
+        return;
+    }
+    const unsigned long long avg = (total + num_ctas - 1) / (unsigned long long)num_ctas;
+    whole = (int)min(avg, 1ull << 30);
+    if (whole < 4) whole = 4;
+    chunk = (int)min((avg + 3) / 4, 1ull << 30);
+    if (chunk < host_chunk) chunk = host_chunk;
+}
+
+// Total work of the call in tiles: every (sequence, KV head) pair's tiles past t_offset.  Summed by the 32 lanes
+// of a warp (the planning kernel sums the same values over its threads).
+__device__ __forceinline__ unsigned long long dec_total_warp(const DecodeArgs &a, int lane) {
+    unsigned long long part = 0;
+    for (int s = lane; s < a.batch; s += 32) part += (unsigned long long)dec_tiles(a, s, false) * a.num_kv_heads;
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    return part;
+}
+
 // Output rows of (sequence s, KV head kvh) from its part_base partials alone (no tile of its own): the
 // element loop is strided over `nthreads` threads starting at `t0`.
 __device__ void plan_merge_bare(const DecodeArgs &a, int s, int kvh, int t0, int nthreads) {
@@ -209,21 +239,8 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
     if ((tid & 31) == 0) atomicAdd(&s_total, part);
     __syncthreads();
-    // split rule: pairs up to the average per-CTA load stay whole; longer ones are cut into pieces of a
-    // quarter of it (never finer than the host's chunk, which sized the partial slots; an eighth measured 2 us
-    // slower at long context: more partials to merge, and the tail pieces already even out the ends)
     int whole, chunk;
-    const int host_chunk = a.plan.chunk / kTile;
-    if (a.plan.fixed) {
-        whole = 0;
-        chunk = host_chunk;
-    } else {
-        const unsigned long long avg = (s_total + num_ctas - 1) / (unsigned long long)num_ctas;
-        whole = (int)min(avg, 1ull << 30);
-        if (whole < 4) whole = 4;
-        chunk = (int)min((avg + 3) / 4, 1ull << 30);
-        if (chunk < host_chunk) chunk = host_chunk;
-    }
+    dec_cut(a, s_total, num_ctas, whole, chunk);
     // Item order: slots 0 .. n_first-1 hold the first split of pairs 0 .. n_first-1 (CTA c's first item, which
     // its producer starts loading before this table exists), then every other item longest first: count those
     // per length bucket, then exclusive offsets from the longest bucket
@@ -522,6 +539,21 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------ producer --
+        // CTA c < n_first owns the first split of pair c.  For a batch of up to kDecLocalCut sequences the warp
+        // sums the call's work itself and cuts the pair as the planning kernel does (dec_cut on the same
+        // total), so the first item -- its Q rows, all its tiles, the consumers' work on them -- runs while
+        // the planning kernel's table is still being written; only the next item waits for the table.
+        const int n_first = min((int)gridDim.x, a.batch * a.num_kv_heads);
+        int4 d_first = make_int4(-1, 0, 0, 0);   // the item the planning kernel writes into slot c, or none
+        if ((int)blockIdx.x < n_first && a.batch <= kDecLocalCut) {
+            int whole, chunk;
+            dec_cut(a, dec_total_warp(a, lane), (int)gridDim.x, whole, chunk);
+            const int s0 = blockIdx.x / a.num_kv_heads, kvh0 = blockIdx.x % a.num_kv_heads;
+            const SplitGeom g = dec_split_geom(dec_tiles(a, s0, false), whole, chunk);
+            if (g.n > 0)   // {s, kvh, t_offset, end of the first split}
+                d_first = make_int4(s0, kvh0, a.t_offset,
+                                    g.n == 1 ? dec_ctx(a, s0) : a.t_offset + dec_split_begin(g, chunk, 1) * kTile);
+        }
         // One thread.  The next item's index is taken when three tiles of the current item remain to be
         // issued (not earlier: an item taken early is held back from idle CTAs) and its record is read a tile
         // later, so both latencies run under the copies already in the ring.  (Reading each tile's block ids
@@ -561,45 +593,30 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 }
             };
-            // CTA c < n_first owns the first split of pair c, which begins at t_offset whatever the plan cuts:
-            // its Q rows and first tiles are requested before the planning kernel's table exists.  They are
-            // inputs the planning kernel does not write (a fused store's new token lies past them), and never
-            // more tiles than any first split of the pair can have: all of a pair of at most 4 tiles (never
-            // split: the plan keeps pairs up to the per-CTA average, at least 4 tiles, whole), 2 of a longer
-            // one (a first chunk has at least 4, a first tail piece at least 2), the chunk when the caller
-            // fixed the split count; at most one ring's worth.
-            const int n_first = min((int)gridDim.x, a.batch * a.num_kv_heads);
-            int npre = 0;
-            if ((int)blockIdx.x < n_first) {
-                const int s0 = blockIdx.x / a.num_kv_heads, kvh0 = blockIdx.x % a.num_kv_heads;
-                const int tiles0 = dec_tiles(a, s0, false);
-                if (tiles0 > 0) {
-                    const int ctx0 = dec_ctx(a, s0);
-                    const int before_new = (ctx0 - 1 - a.t_offset) / kTile;   // tiles before the new token's
-                    const int split_min = a.plan.fixed ? a.plan.chunk / kTile : (tiles0 <= 4 ? tiles0 : 2);
-                    npre = min(min(C::kStages, before_new), split_min);
-                }
-                if (npre > 0) {
-                    mbar_expect_tx(smem_u32(qfull), qbytes);   // the arrival comes with the item, after the table
-                    bulk_load(qsm, q_rows(s0, kvh0), qbytes, smem_u32(qfull));
-                    for (int t = 0; t < npre; ++t)
-                        load_tile(a.block_table + (int64_t)s0 * a.bt_stride, kvh0, a.t_offset + t * kTile, dec_ctx(a, s0), t);
-                    gt = (uint32_t)npre;
-                }
-            }
-            bool pre = npre > 0;
-            asm volatile("griddepcontrol.wait;" ::: "memory");   // the planning kernel's table is complete
             DecPlanHdr *hdr = reinterpret_cast<DecPlanHdr *>(a.plan_ws);
             const int4 *items = reinterpret_cast<const int4 *>(reinterpret_cast<const char *>(a.plan_ws) + kPlanHdrBytes);
-            const int n_items = __ldcg(&hdr->n_items);
             const int4 kEnd = make_int4(-1, 0, 0, 0);
-            // the first item is this CTA's own slot (if it has one); the rest come from the counter
-            int idx = (int)blockIdx.x < n_first ? (int)blockIdx.x : atomicAdd(&hdr->counter, 1);
-            int4 d = idx < n_items ? __ldcg(items + idx) : kEnd;
+            int n_items = 0;
+            bool waited = false;
+            auto wait_table = [&]() {   // the planning kernel's table is complete
+                if (waited) return;
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                n_items = __ldcg(&hdr->n_items);
+                waited = true;
+            };
+            int4 d = d_first;
+            int idx = 0;
+            if (d.x < 0) {
+                // the first item is this CTA's own slot (if it has one); the rest come from the counter
+                wait_table();
+                idx = (int)blockIdx.x < n_first ? (int)blockIdx.x : atomicAdd(&hdr->counter, 1);
+                d = idx < n_items ? __ldcg(items + idx) : kEnd;
+            }
             while (ok) {
                 const int qs = nqi & 1;
                 if (nqi >= 2 && !mbar_wait(smem_u32(qempty + qs), ((nqi >> 1) - 1) & 1, a.dev_error)) break;
                 if (d.x == kDecSkip) {            // a first slot whose pair has no work
+                    wait_table();
                     idx = atomicAdd(&hdr->counter, 1);
                     d = idx < n_items ? __ldcg(items + idx) : kEnd;
                     continue;
@@ -615,20 +632,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                 desc[qs] = d;                     // the item rides in the Q slot's descriptor
                 const int s = d.x, kvh = d.y & 0xffff, t_begin = d.z, t_end = d.w;
                 const int ntiles = (t_end - t_begin + kTile - 1) / kTile;
-                int t_start = 0;
-                if (pre) {
-                    // this is pair blockIdx.x's first split (its slot), whose Q rows and first tiles are on their
-                    // way: the arrival completes the Q slot with the item written
-                    pre = false;
-                    mbar_arrive(smem_u32(qfull + qs));
-                    t_start = npre;
-                } else {
-                    mbar_arrive_expect_tx(smem_u32(qfull + qs), qbytes);
-                    bulk_load(qsm + qs * qslot, q_rows(s, kvh), qbytes, smem_u32(qfull + qs));
-                }
+                mbar_arrive_expect_tx(smem_u32(qfull + qs), qbytes);
+                bulk_load(qsm + qs * qslot, q_rows(s, kvh), qbytes, smem_u32(qfull + qs));
                 ++nqi;
                 const int32_t *bt = a.block_table + (int64_t)s * a.bt_stride;
-                for (int t = t_start; t < ntiles; ++t, ++gt) {
+                for (int t = 0; t < ntiles; ++t, ++gt) {
                     const int st = gt % C::kStages;
                     if (gt >= (uint32_t)C::kStages &&
                         !mbar_wait(smem_u32(empty + st), ((gt / C::kStages) & 1) ^ 1, a.dev_error)) {
@@ -637,13 +645,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                     load_tile(bt, kvh, t_begin + t * kTile, t_end, st);
                     // the next item: index and record, issued now and used when this item's copies are out
-                    if (t == max(t_start, ntiles - 3)) idx_next = atomicAdd(&hdr->counter, 1);
-                    if (t == max(t_start, ntiles - 2)) d_next = idx_next < n_items ? __ldcg(items + idx_next) : kEnd;
-                }
-                // an item whose every tile was loaded before the table (one tile) still takes the next item
-                if (t_start >= ntiles) {
-                    idx_next = atomicAdd(&hdr->counter, 1);
-                    d_next = idx_next < n_items ? __ldcg(items + idx_next) : kEnd;
+                    if (t == max(0, ntiles - 3)) {
+                        wait_table();
+                        idx_next = atomicAdd(&hdr->counter, 1);
+                    }
+                    if (t == max(0, ntiles - 2)) d_next = idx_next < n_items ? __ldcg(items + idx_next) : kEnd;
                 }
                 d = d_next;
             }

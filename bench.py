@@ -341,7 +341,7 @@ def bench_primary(args, world, rank, device, pk):
         "kv_hbm_frac_of_measured": case.kv_bytes_read() / step_mean / 1e9 / pk["hbm_gbs"],
         "kv_hbm_frac_of_8tbs": case.kv_bytes_read() / step_mean / 1e9 / 8000.0,
         "store_decode_us": step_mean * 1e6, "step_us_median": statistics.median(t_step) * 1e6,
-        "roofline": {"kernel": "decode_split_kernel<128> (store fused)", "bound": "hbm",
+        "roofline": {"kernel": "decode_split_kernel<128, 1> (store fused)", "bound": "hbm",
                      "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                      "traffic": recorded_traffic("store_decode_qwen3_0.6b"), "alg_bytes_per_launch": alg},
         # per step: the kernels of one pa_store_kv_decode call (planning, decode with the store fused in, and a
@@ -505,7 +505,7 @@ def bench_secondary(args, device, pk, names):
         "store_prefill_fused_us": tfm * 1e6, "store_prefill_fused_tflops": fl / tfm / 1e12,
         "tflops": ach, "new_tokens": case.total_q, "prefill_tokens_per_s": case.total_q / (tpm + tsm),
         "store_gbps": store_bytes / tsm / 1e9,
-        "roofline": {"kernel": "prefill_kernel<128>", "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
+        "roofline": {"kernel": "prefill_kernel<128, 0, 0>", "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
                      "frac_of_sustained": ach / pk["bf16_tflops_sustained"],
                      "traffic": recorded_traffic("prefill_varlen")},
